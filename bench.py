@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Benchmark of the 2:4 sparse path on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole path over one batch of synthetic input:
+  bf16 workloads:  [Wanda: column norms] -> prune (3:4 stage for the
+                   progressive workload) -> fused prune+compress 2:4 ->
+                   sparse GEMM Y = X * W'^T
+  int8 workload:   prune 2:4 -> per-channel scale -> compress to int8 ->
+                   per-tensor activation scale -> quantise X -> int8 sparse
+                   GEMM with bf16 dequantisation.
+`value` = dense-equivalent TFLOP/s of the GEMM (2*M*N*K per step) over the
+whole step time; per-kernel figures and the roofline of the dominant kernel
+(the GEMM) are reported beside it.  Inputs are resident in HBM; L2 (126 MB)
+is flushed between timed steps by writing a 512 MB buffer.
+
+Multi-GPU: one process per GPU (torchrun), each rank runs an independent
+replica of the workload (weak scaling); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from structured_sparse_gemm_sp24_b200 import inputs as I  # noqa: E402
+from structured_sparse_gemm_sp24_b200 import sp24 as B  # noqa: E402
+
+METRIC = "2:4 sparse GEMM dense-equiv TFLOP/s & % sparse TC peak; prune+compress GB/s"
+DEFAULT_WORKLOAD = "bert_fc1"
+SPARSE_RATIO = 2.0          # nominal sparse / dense tensor throughput (4.5 / 2.25 PF)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+# --------------------------------------------------------------------- peaks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# -------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every ~20 ms (read only)."""
+
+    REASONS = {
+        0x0000000000000001: "gpu_idle", 0x0000000000000002: "applications_clocks_setting",
+        0x0000000000000004: "sw_power_cap", 0x0000000000000008: "hw_slowdown",
+        0x0000000000000010: "sync_boost", 0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown", 0x0000000000000080: "hw_power_brake_slowdown",
+        0x0000000000000100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        n = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM))
+                r = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------- workload
+class Runner:
+    """Device buffers for one workload and the calls of one step."""
+
+    def __init__(self, wl: I.Workload, device):
+        self.wl = wl
+        self.dev = device
+        self.N, self.K, self.M = wl.N, wl.K, wl.M
+        d = device
+        self.W = wl.W.to(d)
+        self.X = wl.X.to(d)
+        self.Xc = wl.Xc.to(d) if wl.Xc is not None else None
+        N, K, M = self.N, self.K, self.M
+        self.mask1 = torch.empty((N, K // 8), dtype=torch.uint8, device=d)
+        self.mask2 = torch.empty((N, K // 8), dtype=torch.uint8, device=d)
+        self.ws = torch.empty(max(B.sp24_prune_workspace_bytes(K, B.SP24_WANDA), 16),
+                              dtype=torch.uint8, device=d)
+        vdt = torch.int8 if wl.int8 else torch.bfloat16
+        self.vals = torch.empty((N, K // 2), dtype=vdt, device=d)
+        self.meta = torch.empty(B.sp24_meta_bytes(N, K), dtype=torch.uint8, device=d)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=d)
+        if wl.int8:
+            self.s_w = torch.empty(N, dtype=torch.float32, device=d)
+            self.s_x = torch.empty(4, dtype=torch.float32, device=d)
+            self.act_ws = torch.empty(B.sp24_act_scale_workspace_bytes(), dtype=torch.uint8,
+                                      device=d)
+            self.Xq = torch.empty((M, K), dtype=torch.int8, device=d)
+        self.wanda = wl.mode == "wanda"
+
+    # number of library kernel launches per step (see the calls below)
+    def launches_per_step(self) -> int:
+        if self.wl.int8:
+            return 1 + 1 + 1 + 7 + 1 + 1     # prune, wscale, compress, act_scale, quantize, gemm
+        if self.wanda and self.wl.progressive:
+            return 2 + 1 + 1                 # colnorm+prune(3:4), prune_compress, gemm
+        if self.wanda:
+            return 2 + 1 + 1
+        return 1 + 1                         # prune_compress, gemm
+
+    def step(self, ev=None):
+        """Enqueues one step; `ev` = list of 4 events: start, after pruning,
+        after compression, after the GEMM."""
+        rec = (lambda i: ev[i].record()) if ev else (lambda i: None)
+        wl = self.wl
+        rec(0)
+        if wl.int8:
+            B.sp24_prune(self.W, None, B.SP24_MAGNITUDE, 2, None, self.mask2, None)
+            B.sp24_wscale(self.W, self.mask2, 0.9999, self.s_w)
+            rec(1)
+            B.sp24_compress(self.W, self.mask2, B.SP24_INT8, self.s_w, self.vals, self.meta)
+            B.sp24_act_scale(self.X, 0.9999, self.s_x, self.act_ws)
+            B.sp24_quantize(self.X, self.s_x, self.Xq)
+            rec(2)
+            B.sp24_gemm(self.Xq, self.vals, self.meta, self.N, B.SP24_INT8, self.s_x, self.s_w,
+                        B.SP24_OUT_BF16, None, self.Y)
+        elif self.wanda:
+            # prune also leaves the float64 column norms in its workspace
+            n_keep = 3 if wl.progressive else 2
+            B.sp24_prune(self.W, self.Xc, B.SP24_WANDA, n_keep, None, self.mask1, self.ws)
+            rec(1)
+            B.sp24_prune_compress(self.W, B.SP24_WANDA, self.ws,
+                                  self.mask1 if wl.progressive else None, None, B.SP24_BF16,
+                                  None, self.vals, self.meta)
+            rec(2)
+            B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
+                        B.SP24_OUT_BF16, None, self.Y)
+        else:
+            rec(1)
+            B.sp24_prune_compress(self.W, B.SP24_MAGNITUDE, None, None, None, B.SP24_BF16, None,
+                                  self.vals, self.meta)
+            rec(2)
+            B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
+                        B.SP24_OUT_BF16, None, self.Y)
+        rec(3)
+
+    def flops(self) -> float:
+        return 2.0 * self.M * self.N * self.K
+
+    def gemm_bytes(self) -> float:
+        """Algorithmic bytes of one GEMM launch: X + values + metadata + Y."""
+        N, K, M = self.N, self.K, self.M
+        if self.wl.int8:
+            return M * K + N * K / 2 + N * K / 8 + 2 * M * N + 4 * N
+        return 2 * M * K + N * K + N * K / 8 + 2 * M * N
+
+    def compress_bytes(self) -> float:
+        """Algorithmic bytes of the compression stage (fused prune+compress for
+        bf16: read W, write values + metadata)."""
+        N, K = self.N, self.K
+        if self.wl.int8:
+            # compress int8: read W + mask, write values + metadata; act scale
+            # passes and quantisation are reported in the same stage
+            return 2 * N * K + N * K / 8 + N * K / 2 + N * K / 8
+        extra = N * K / 8 if self.wl.progressive else 0   # mask_in
+        return 2 * N * K + extra + N * K + N * K / 8
+
+    def prune_bytes(self) -> float:
+        N, K = self.N, self.K
+        if self.wl.int8:
+            return 2 * N * K + N * K / 8 + (2 * N * K + N * K / 8 + 4 * N)   # prune + wscale
+        if self.wanda:
+            mc = self.wl.Xc.shape[0]
+            return 2 * mc * K + 8 * K + 2 * N * K + 8 * K + N * K / 8
+        return 0.0
+
+    def h2d_inputs(self):
+        t = [self.wl.W, self.wl.X]
+        if self.wl.Xc is not None:
+            t.append(self.wl.Xc)
+        return t
+
+
+def time_steps(runner, steps, flush, stream):
+    """Per-step CUDA events (L2 flushed before each step, outside the events)."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        runner.step(evs[i])
+    torch.cuda.synchronize()
+    tot = [e[0].elapsed_time(e[3]) for e in evs]
+    prune = [e[0].elapsed_time(e[1]) for e in evs]
+    comp = [e[1].elapsed_time(e[2]) for e in evs]
+    gemm = [e[2].elapsed_time(e[3]) for e in evs]
+    return tot, prune, comp, gemm
+
+
+def time_e2e(runner, steps, device):
+    """Same step through host buffers: pinned H2D copies of the step's inputs and
+    a D2H copy of Y inside the timed region."""
+    host_in = [t.pin_memory() for t in runner.h2d_inputs()]
+    dev_in = [runner.W, runner.X] + ([runner.Xc] if runner.Xc is not None else [])
+    host_y = torch.empty(runner.Y.shape, dtype=runner.Y.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_y.numel() * host_y.element_size()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        for hd, dd in zip(host_in, dev_in):
+            dd.copy_(hd, non_blocking=True)
+        runner.step()
+        host_y.copy_(runner.Y, non_blocking=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(steps):
+        for hd, dd in zip(host_in, dev_in):
+            dd.copy_(hd, non_blocking=True)
+        runner.step()
+        host_y.copy_(runner.Y, non_blocking=True)
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps, h2d, d2h
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(wl: I.Workload, budget_s: float):
+    """Times the CPU oracle (as it stands) on a bounded sample of the workload:
+    the full prune + compress of W, then the GEMM on as many X rows as fit the
+    budget.  Returns (dense-equivalent flops processed, seconds, description)."""
+    from oracle import sp24_oracle as O
+    import threadpoolctl
+
+    w = wl.W.to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    if wl.int8:
+        keep = O.prune(w, O.MAGNITUDE, 2)
+        s_w = O.channel_scales(w, keep)
+        vals, meta = O.compress(O.quantize(w, s_w[:, None]), keep)
+    else:
+        xc = wl.Xc.to(torch.float64).numpy() if wl.Xc is not None else None
+        mode = O.WANDA if wl.mode == "wanda" else O.MAGNITUDE
+        if wl.progressive:
+            keep = O.progressive(w, mode, xc)[1]
+        else:
+            keep = O.prune(w, mode, 2, xc=xc)
+        vals, meta = O.compress(w, keep)
+    t_conv = time.perf_counter() - t0
+    rows, t_gemm, r = 0, 0.0, 8
+    while rows < wl.M and t_conv + t_gemm < budget_s:
+        r = min(r, wl.M - rows)
+        t1 = time.perf_counter()
+        if wl.int8:
+            x = wl.X[rows:rows + r].numpy()
+            s_x = O.tensor_scale(x)   # per-sample scale: same arithmetic, bounded cost
+            acc = O.gemm_int8_acc(O.quantize(x, s_x), vals, meta, wl.K)
+            O.dequant_bf16(acc, s_x, s_w)
+        else:
+            O.gemm(wl.X[rows:rows + r].to(torch.float64).numpy(), vals, meta, wl.K)
+        t_gemm += time.perf_counter() - t1
+        rows += r
+        r *= 2
+    cores = None
+    for info in threadpoolctl.threadpool_info():
+        cores = max(cores or 0, int(info.get("num_threads", 0)))
+    sample = (f"full prune+compress of W {wl.N}x{wl.K} ({t_conv:.2f}s) + GEMM on {rows} of "
+              f"{wl.M} X rows ({t_gemm:.2f}s); flops scaled by rows")
+    return 2.0 * rows * wl.N * wl.K, t_conv + t_gemm, sample, cores or os.cpu_count()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = I.by_name(args.workload)
+    per_step = []
+    sample = ""
+    cores = os.cpu_count()
+    budget = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup + args.steps):
+        flops, secs, sample, cores = oracle_sample(wl, budget)
+        if i >= args.warmup:
+            per_step.append((flops, secs))
+    flops = sum(f for f, _ in per_step)
+    secs = sum(s for _, s in per_step)
+    value = flops / secs / 1e12
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / max(1, len(per_step)), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sp24", choices=["sp24", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+    B.lib()
+
+    wl = I.by_name(args.workload)
+    runner = Runner(wl, device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        flush.zero_()
+        runner.step()
+    torch.cuda.synchronize()
+    if B.sp24_device_status() != B.SP24_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    barrier()
+    with ClockSampler(local) as clk:
+        tot, prune, comp, gemm = time_steps(runner, args.steps, flush, stream)
+    barrier()
+    total_ms = sum(tot)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * args.steps * runner.flops() / (total_ms * 1e-3) / 1e12
+
+    e2e_ms, h2d, d2h = time_e2e(runner, max(3, min(args.steps, 50)), device)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * runner.flops() / (e2e_ms * 1e-3) / 1e12
+    if B.sp24_device_status() != B.SP24_OK:
+        raise SystemExit("device status not OK after timing")
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return 0
+
+    peaks = load_peaks()
+    sparse_peak = SPARSE_RATIO * peaks["bf16_tflops"]
+    if wl.int8:
+        sparse_peak *= 2.0   # int8 tensor rate = 2x bf16 (nominal)
+    gemm_ms = statistics.mean(gemm)
+    comp_ms = statistics.mean(comp)
+    prune_ms = statistics.mean(prune)
+    g_tflops = runner.flops() / (gemm_ms * 1e-3) / 1e12
+    g_gbs = runner.gemm_bytes() / (gemm_ms * 1e-3) / 1e9
+    t_tensor = runner.flops() / (sparse_peak * 1e12)
+    t_hbm = runner.gemm_bytes() / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tensor >= t_hbm else "hbm"
+    if bound == "tensor":
+        roof = {"bound": "tensor", "achieved": g_tflops, "peak": sparse_peak, "unit": "TFLOP/s",
+                "frac": g_tflops / sparse_peak}
+    else:
+        roof = {"bound": "hbm", "achieved": g_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": g_gbs / peaks["hbm_gbs"]}
+    roof["traffic"] = None
+    roof["peak_source"] = peaks["source"] + (" (2x dense bf16 burst)" if not wl.int8 else
+                                             " (4x dense bf16 burst)")
+    roof["kernel"] = "gemm_sp_kernel"
+    c_gbs = runner.compress_bytes() / (comp_ms * 1e-3) / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8" if wl.int8 else "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K,
+                   "mode": wl.mode, "progressive": wl.progressive,
+                   "l2": "flushed between steps (512 MB write)", "parallelism": f"replicas{world}"},
+        "gemm": {"ms": gemm_ms, "tflops_dense_equiv": g_tflops, "gbs": g_gbs,
+                 "frac_sparse_peak": g_tflops / sparse_peak},
+        "prune_compress": {"ms": comp_ms, "gbs": c_gbs, "frac_hbm": c_gbs / peaks["hbm_gbs"],
+                           "prune_ms": prune_ms},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": runner.launches_per_step() * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        flops, secs, sample, cores = oracle_sample(wl, args.cpu_budget)
+        line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

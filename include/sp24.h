@@ -1,0 +1,220 @@
+/*
+ * sp24.h -- C ABI of libsp24: 2:4 fine-grained structured sparsity on B200.
+ *
+ * Three verbs, each an asynchronous launch on a caller stream:
+ *   prune    W (+ calibration rows)          -> keep mask     (N:4, n_keep of 4)
+ *   compress W + mask (+ INT8 scales)        -> values + metadata (tcgen05 operand layout)
+ *   gemm     X, values, metadata (+ scales)  -> Y = X * W'^T
+ * plus the INT8 calibration helpers (per-channel / per-tensor scales,
+ * activation quantisation) and status queries.
+ *
+ * Sources ("pages") are cited by title and section:
+ *   [Ampere-sparsity] NVIDIA x Tencent MLPD article on Ampere fine-grained
+ *       structured sparsity (nvidia.zhidx.com): 2:4 pattern and compressed
+ *       format (Figure 1), progressive sparsity (Figures 3-4), "PTQ and QAT".
+ *   [Wanda-2:4] "Structured Pruning: 2:4 sparse inference with the Wanda
+ *       algorithm" (zyxy.net), sections 1.3, 2.1, 2.2.
+ *   [Sparse-accel forum] oeforum.com post on sparse acceleration (2-bit
+ *       metadata, offline conversion, INT8 x 2:4).
+ *   [Orin ch.7] "Chapter 7: 2:4 Structured Sparsity" (Orin NN design book),
+ *       sections 2.1 (worked example), 2.3 (alignment), 6.1 (every 1x4 block
+ *       must be valid or the sparse path silently falls back), 6.2 (padding).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named W, X, Xc, mask*, vals, meta, norms, s_*, Y and workspace are
+ *   DEVICE pointers owned by the caller; the library never allocates, frees or
+ *   keeps them.  Matrices are row-major and densely packed (row stride = number
+ *   of columns).  Every device pointer must be 16-byte aligned (cudaMalloc
+ *   gives 256) or the call returns SP24_ERR_ALIGN.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Every call only enqueues work; it does not synchronise.
+ * - Argument, size and alignment errors are detected on the host before any
+ *   launch and returned synchronously; nothing is enqueued in that case.
+ * - Errors found on the device (a group that does not keep exactly two
+ *   positions, a bounded wait that gave up) are recorded in a per-device
+ *   status word and reported by sp24_device_status().
+ * - bf16 means IEEE-754 binary32 truncated to its top 16 bits (bfloat16); the
+ *   library reads inputs as bit patterns and assumes finite values.
+ * - Weight layout: W[N][K], N = output channels, K = input channels; groups of
+ *   4 run along K ([Orin ch.7] 2.1).  A 1x1 convolution over NHWC activations
+ *   is the same GEMM with M = batch*H*W and K = C_in ([Orin ch.7] 2.2).
+ */
+#ifndef SP24_H_
+#define SP24_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sp24_status {
+    SP24_OK = 0,
+    SP24_ERR_ARG = 1,         /* null pointer, negative size, unknown enum value */
+    SP24_ERR_ALIGN = 2,       /* a size or pointer breaks an alignment rule */
+    SP24_ERR_PATTERN = 3,     /* a group of 4 does not keep exactly two positions */
+    SP24_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+    SP24_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
+    SP24_ERR_UNSUPPORTED = 6  /* no sm_100 device, or a combination not provided */
+} sp24_status;
+
+/* scoring modes for sp24_prune */
+enum { SP24_MAGNITUDE = 0, SP24_WANDA = 1 };
+/* value types of the compressed weight and of X in sp24_gemm */
+enum { SP24_BF16 = 0, SP24_INT8 = 1 };
+/* output kinds of sp24_gemm */
+enum { SP24_OUT_BF16 = 0, SP24_OUT_INT32 = 1, SP24_OUT_INT8 = 2 };
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Bytes of a keep mask for W[N][K]: one nibble per group of 4 (bit p set when
+ * position p is kept), group 2b in the low nibble of byte b; N*K/8.
+ * K must be a multiple of 8.  Returns 0 for invalid sizes. */
+size_t sp24_mask_bytes(int64_t N, int64_t K);
+
+/* Bytes of the compressed values: N rows of K/2 kept values, in ascending
+ * position order within each group ([Ampere-sparsity] Figure 1:
+ * only the nonzeros are stored, 50 % of the value bytes).
+ * dtype SP24_BF16 -> 2 bytes each, SP24_INT8 -> 1 byte each. */
+size_t sp24_vals_bytes(int64_t N, int64_t K, int dtype);
+
+/* Bytes of the metadata: 2 bits per kept value = 4 bits per group
+ * ([Sparse-accel forum]; [Orin ch.7] 2.1 "Metadata (2-bit)"), stored in the
+ * tcgen05.mma.sp operand layout: chunks of 128 rows x 128 K-positions
+ * (2048 bytes), N rounded up to 128 and K rounded up to 128.
+ * The layout depends on dtype but the size does not. */
+size_t sp24_meta_bytes(int64_t N, int64_t K);
+
+/* Scratch bytes sp24_prune needs for `mode`: 8*K (float64 column norms) for
+ * SP24_WANDA, 0 for SP24_MAGNITUDE. */
+size_t sp24_prune_workspace_bytes(int64_t K, int mode);
+
+/* ------------------------------------------------------------- pruning */
+
+/* Wanda activation statistic ([Wanda-2:4] 2.1): norms[j] = sqrt(sum_t Xc[t][j]^2)
+ * over the Mc calibration rows, float64, summed sequentially in t (each
+ * square of a bf16 value is exact in float64; one rounding per addition).
+ * Xc: bf16 [Mc][K].  norms: float64 [K].  Mc >= 1, K >= 1, K % 8 == 0. */
+sp24_status sp24_colnorm(const void* Xc, int64_t Mc, int64_t K, double* norms,
+                         void* stream);
+
+/* N:4 pruning along K ([Wanda-2:4] 1.3 and 2.2; [Orin ch.7] 2.1 Step 1):
+ * within each group of 4 consecutive weights of a row, keep the n_keep
+ * positions of largest score; position p is kept iff fewer than n_keep others
+ * beat it, q beating p when s_q > s_p or (s_q == s_p and q < p).
+ *   mode SP24_MAGNITUDE: s = |w|
+ *   mode SP24_WANDA:     s = |w| * norms[j] in float64, norms from Xc as in
+ *                        sp24_colnorm, computed into `workspace`
+ * n_keep = 3 is the 25 % stage of progressive sparsity, n_keep = 2 the 50 %
+ * stage ([Ampere-sparsity] Figure 4).  With mask_in != NULL the weights
+ * dropped by mask_in score 0 (the second stage recomputes the mask on the
+ * remaining weights).
+ *   W: bf16 [N][K].  Xc: bf16 [Mc][K] (SP24_WANDA only, else ignored).
+ *   mask_in (nullable), mask_out: sp24_mask_bytes(N, K) bytes.
+ *   workspace: sp24_prune_workspace_bytes(K, mode) bytes (NULL if 0).
+ * Rules: N >= 0, K % 8 == 0, n_keep in {2, 3}; Mc >= 1 for SP24_WANDA. */
+sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc,
+                       int64_t Mc, int mode, int n_keep, const uint8_t* mask_in,
+                       uint8_t* mask_out, void* workspace, void* stream);
+
+/* --------------------------------------------------------- INT8 scales */
+
+/* Per-output-channel weight scale ([Ampere-sparsity] "PTQ and QAT": the scale
+ * covers `coverage` (0.9999) of the values): t_n = the r-th smallest |W[n][k]|
+ * over the c kept positions of row n, r = max(1, ceil(coverage * c)) computed
+ * in IEEE double; s_w[n] = float(t_n) / 127.0f (float32 divide), or 1 when
+ * t_n == 0.  For c <= 9999 and coverage 0.9999 this is the row maximum.
+ *   W: bf16 [N][K].  mask: sp24_mask_bytes(N, K) bytes.  s_w: float32 [N].
+ * Rules: K % 8 == 0, 0 < coverage <= 1, K/2 <= 65536. */
+sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K,
+                        double coverage, float* s_w, void* stream);
+
+/* Per-tensor activation scale: t = the r-th smallest |X[i]| over all `count`
+ * float32 values, r = max(1, ceil(coverage * count)) in IEEE double;
+ * *s_x = t / 127.0f (float32), or 1 when t == 0.  Exact (radix selection on
+ * the float32 bit patterns).
+ *   X: float32 [count].  s_x: one float32 (device).
+ *   workspace: sp24_act_scale_workspace_bytes() bytes.
+ * Rules: count >= 1, 0 < coverage <= 1. */
+size_t sp24_act_scale_workspace_bytes(void);
+sp24_status sp24_act_scale(const float* X, int64_t count, double coverage,
+                           float* s_x, void* workspace, void* stream);
+
+/* Symmetric quantisation: Xq[i] = clamp(rint(X[i] / *s_x), -127, 127) with an
+ * IEEE float32 divide and round-half-to-even.
+ *   X: float32 [count].  s_x: one float32 (device).  Xq: int8 [count]. */
+sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x,
+                          int8_t* Xq, void* stream);
+
+/* ---------------------------------------------------------- compression */
+
+/* Compression ([Ampere-sparsity] Figure 1; [Orin ch.7] 2.1 Step 2): for each
+ * group with kept positions lo < hi, vals gets W[lo] then W[hi] and the
+ * metadata records the two 2-bit positions.
+ *   dtype SP24_BF16: vals bf16 [N][K/2] (the weights' own bits).
+ *   dtype SP24_INT8: vals int8 [N][K/2], q = clamp(rint(W / s_w[n]), -127, 127)
+ *                    with a float32 divide (s_w from sp24_wscale).
+ *   meta: sp24_meta_bytes(N, K) bytes in the operand layout of
+ *         tcgen05.mma.sp for `dtype` (opaque to callers; rows >= N and
+ *         positions >= K are filled with a valid pattern over zero values).
+ * A group whose mask nibble does not have exactly two bits set is a pattern
+ * error ([Orin ch.7] 6.1): it is reported by sp24_device_status() as
+ * SP24_ERR_PATTERN (never silently treated as dense); its outputs are
+ * unspecified.
+ * Rules: K % 8 == 0 (SP24_BF16: K % 16 == 0; SP24_INT8: K % 32 == 0, so that
+ * value rows stay 16-byte aligned); s_w required for SP24_INT8. */
+sp24_status sp24_compress(const void* W, const uint8_t* mask, int64_t N, int64_t K,
+                          int dtype, const float* s_w, void* vals, void* meta,
+                          void* stream);
+
+/* Fused prune + compress in one pass over W: the mask of sp24_prune (with
+ * n_keep = 2) and the outputs of sp24_compress.  mask_out may be NULL.
+ * norms: float64 [K] from sp24_colnorm for SP24_WANDA, else NULL. */
+sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
+                                const double* norms, const uint8_t* mask_in,
+                                uint8_t* mask_out, int dtype, const float* s_w,
+                                void* vals, void* meta, void* stream);
+
+/* ----------------------------------------------------------- sparse GEMM */
+
+/* Y = X * W'^T with W' the 2:4 weight given by (vals, meta) ([Orin ch.7] 2.1
+ * Step 3: only the kept weights are multiplied, each with the activation its
+ * 2-bit position selects; [Sparse-accel forum]: INT8 x 2:4).
+ *   dtype SP24_BF16: X bf16 [M][K]; fp32 accumulation; out_kind SP24_OUT_BF16
+ *       writes Y bf16 [M][N] = rne(acc).  s_x, s_w, s_y ignored (may be NULL).
+ *   dtype SP24_INT8: X int8 [M][K] (from sp24_quantize); int32 accumulation,
+ *       exact.  out_kind SP24_OUT_INT32: Y int32 [M][N] = acc.
+ *       SP24_OUT_BF16: Y bf16 = rne(float(acc) * (s_x * s_w[n])), each step
+ *       float32 round-to-nearest, in that order.
+ *       SP24_OUT_INT8: Y int8 = clamp(rint((float(acc) * (s_x * s_w[n])) / s_y),
+ *       -127, 127), float32 divide.
+ *       s_x, s_y: one float32 each (device); s_w: float32 [N] (device).
+ * vals/meta come from sp24_compress with the same dtype, N and K.
+ * Rules: M >= 0, N >= 0, N % 8 == 0; K >= 16, K % 16 == 0 (bf16) or
+ * K % 32 == 0 (int8); alignment of 16 bytes for every pointer.  Ragged M, N
+ * and K tails are handled in the kernel (no padding copies; [Orin ch.7] 6.2). */
+sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
+                      const void* meta, int64_t N, int dtype, const float* s_x,
+                      const float* s_w, int out_kind, const float* s_y, void* Y,
+                      void* stream);
+
+/* --------------------------------------------------------------- status */
+
+/* Synchronises `stream`, then returns and clears the device status word of the
+ * current device (SP24_OK, SP24_ERR_PATTERN or SP24_ERR_TIMEOUT), or
+ * SP24_ERR_CUDA if the stream reports a CUDA error. */
+sp24_status sp24_device_status(void* stream);
+
+/* Static text for a status code (never NULL). */
+const char* sp24_strerror(int status);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int sp24_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP24_H_ */

@@ -1,0 +1,96 @@
+// libsp24: size queries, status word, error strings, device checks.
+#include <mutex>
+
+#include "sp24_device.cuh"
+#include "sp24_host.h"
+
+namespace sp24 {
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_dev_ok[kMaxDevices];   // 0 unknown, 1 sm_100, 2 other
+int g_dev_sms[kMaxDevices];
+std::mutex g_dev_mu;
+}  // namespace
+
+sp24_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SP24_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SP24_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_dev_ok[dev] == 0) {
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return SP24_ERR_CUDA;
+    g_dev_ok[dev] = (major == 10) ? 1 : 2;
+    g_dev_sms[dev] = sms;
+  }
+  return g_dev_ok[dev] == 1 ? SP24_OK : SP24_ERR_UNSUPPORTED;
+}
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDevices || g_dev_sms[dev] == 0) return 148;
+  return g_dev_sms[dev];
+}
+
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" {
+
+size_t sp24_mask_bytes(int64_t N, int64_t K) {
+  if (N < 0 || K < 0 || (K % 8) != 0) return 0;
+  return static_cast<size_t>(N) * static_cast<size_t>(K / 8);
+}
+
+size_t sp24_vals_bytes(int64_t N, int64_t K, int dtype) {
+  if (N < 0 || K < 0 || (K % 8) != 0) return 0;
+  const size_t el = dtype == SP24_BF16 ? 2 : (dtype == SP24_INT8 ? 1 : 0);
+  return static_cast<size_t>(N) * static_cast<size_t>(K / 2) * el;
+}
+
+size_t sp24_meta_bytes(int64_t N, int64_t K) {
+  if (N < 0 || K < 0 || (K % 8) != 0) return 0;
+  const size_t nr = static_cast<size_t>((N + 127) / 128);
+  const size_t kc = static_cast<size_t>((K + 127) / 128);
+  return nr * kc * 2048u;
+}
+
+size_t sp24_prune_workspace_bytes(int64_t K, int mode) {
+  if (K < 0) return 0;
+  return mode == SP24_WANDA ? static_cast<size_t>(K) * sizeof(double) : 0;
+}
+
+sp24_status sp24_device_status(void* stream) {
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SP24_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return SP24_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SP24_ERR_CUDA;
+  }
+  if (word & kErrTimeoutBit) return SP24_ERR_TIMEOUT;
+  if (word & kErrPatternBit) return SP24_ERR_PATTERN;
+  return SP24_OK;
+}
+
+const char* sp24_strerror(int status) {
+  switch (status) {
+    case SP24_OK: return "ok";
+    case SP24_ERR_ARG: return "invalid argument (null pointer, negative size or unknown enum)";
+    case SP24_ERR_ALIGN: return "alignment rule broken (sizes or 16-byte pointer alignment)";
+    case SP24_ERR_PATTERN: return "a group of 4 does not keep exactly two positions";
+    case SP24_ERR_CUDA: return "CUDA runtime error";
+    case SP24_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case SP24_ERR_UNSUPPORTED: return "unsupported device or argument combination";
+    default: return "unknown status";
+  }
+}
+
+int sp24_version(void) { return 100; }
+
+}  // extern "C"

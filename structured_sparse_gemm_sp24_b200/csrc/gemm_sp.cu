@@ -1,0 +1,461 @@
+// libsp24: sparse GEMM Y = X * W'^T on the 5th-generation tensor cores
+// (tcgen05.mma.sp), for bf16 (fp32 accumulate) and int8 (int32 accumulate).
+//
+// [Orin ch.7] "Chapter 7: 2:4 Structured Sparsity" 2.1 Step 3: the sparse
+// tensor core multiplies only the kept weights, each with the activation its
+// 2-bit position selects; [Sparse-accel forum] (oeforum.com): INT8 x 2:4.
+//
+// Operand roles.  The sparse operand of tcgen05.mma.sp is A (the MMA's M
+// side), so the kernel computes one 128 (output channels) x BN (tokens) tile
+// of Y^T = W' * X^T per CTA:
+//   A = compressed W tile: 128 rows x 128 bytes per stage (bf16: 64 values =
+//       128 logical K; int8: 128 values = 256 logical K), TMA, 128B swizzle;
+//   B = X tile: BN rows x 256 bytes per stage as two 128B-swizzled halves;
+//   E = metadata chunk(s) (2048 bytes per 128 logical K), one bulk copy, then
+//       tcgen05.cp into tensor memory, where tcgen05.mma.sp reads it;
+//   D = fp32 / int32 accumulator in tensor memory: lane = output channel,
+//       column = token.
+// Each stage issues 4 MMAs (K = 32 for kind::f16, 64 for kind::i8); both
+// advance A by 32 bytes and B by 64 bytes inside the swizzle atoms.
+//
+// Split-K.  When the output tiles alone cannot fill the GPU (small M: the
+// weight stream is the bound), S CTAs of a thread-block cluster split the K
+// blocks of one tile; their partial accumulators are summed in a fixed order
+// through distributed shared memory, so the result does not depend on timing.
+//
+// Warp roles (128 threads): warp 0 lane 0 issues TMA, warp 1 lane 0 issues
+// tcgen05 (copy + MMA), warp 2 owns the tensor-memory allocation; all four
+// warps run the epilogue (tcgen05.ld of their 32 lanes -> scale / cast ->
+// shared-memory transpose -> coalesced 16-byte stores of Y rows).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "sp24_device.cuh"
+#include "sp24_host.h"
+
+namespace sp24 {
+
+template <int kDtype, int BN, int STAGES>
+struct GemmCfg {
+  static constexpr int kABytes = 128 * 128;                         // A tile per stage
+  static constexpr int kBHalfBytes = BN * 128;                      // one B half
+  static constexpr int kMetaChunks = kDtype == SP24_BF16 ? 1 : 2;   // 2048 B each
+  static constexpr int kEBytes = 2048 * kMetaChunks;
+  static constexpr int kStageBytes = kABytes + 2 * kBHalfBytes + kEBytes;
+  static constexpr int kLogicalK = kDtype == SP24_BF16 ? 128 : 256;  // K per stage
+  static constexpr int kMmaK = kLogicalK / 4;                        // K per MMA
+  static constexpr int kMetaCols = 4 * kMetaChunks;                  // TMEM columns per stage
+  // accumulator columns [0, BN), two metadata buffers after it
+  static constexpr int kMetaCol0 = BN;
+  static constexpr int kTmemNeeded = BN + 2 * kMetaCols;
+  static constexpr int kTmemCols = kTmemNeeded <= 32 ? 32
+                                   : kTmemNeeded <= 64 ? 64
+                                   : kTmemNeeded <= 128 ? 128
+                                   : kTmemNeeded <= 256 ? 256 : 512;
+  // stages are 1024-aligned: A, then the two B halves, then E
+  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kSmemBytes = STAGES * kStageStride + 1024 /*align slack*/ + 256 /*bars*/;
+  static_assert(kTmemNeeded <= 512, "tensor memory overflow");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+  // epilogue staging of a partial tile (fp32/int32, [BN][128]) reuses the ring
+  static_assert(STAGES * kStageStride >= BN * 128 * 4, "staging does not fit");
+};
+
+// Instruction descriptor of tcgen05.mma.sp (M = 128, K-major A and B).
+template <int kDtype, int BN>
+__device__ __forceinline__ uint32_t make_idesc(uint32_t id2) {
+  const uint32_t c_fmt = kDtype == SP24_BF16 ? 1u : 2u;  // F32 : S32
+  const uint32_t ab_fmt = 1u;                             // BF16 : signed int8
+  return (id2 & 3u) | (1u << 2) | (c_fmt << 4) | (ab_fmt << 7) | (ab_fmt << 10) |
+         (static_cast<uint32_t>(BN >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+struct GemmArgs {
+  const uint8_t* meta;
+  const float* s_x;
+  const float* s_w;
+  const float* s_y;
+  void* y;
+  int64_t m, n, k;
+  int kblocks;        // stages over the whole K
+  int kb_per_split;   // stages per split CTA
+  int out_kind;
+};
+
+template <int kDtype, int BN, int STAGES, int SPLIT>
+__global__ void __launch_bounds__(128, 1)
+gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
+               const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  using C = GemmCfg<kDtype, BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageStride);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* accum_bar = empty_bar + STAGES;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_bar + 1);
+  uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t split = SPLIT > 1 ? cluster_ctarank() : 0u;
+  const int64_t row_tile = blockIdx.y;
+  const int64_t tok_tile = blockIdx.z;
+  const int kb_begin = static_cast<int>(split) * args.kb_per_split;
+  int kb_end = kb_begin + args.kb_per_split;
+  if (kb_end > args.kblocks) kb_end = args.kblocks;
+  const int n_iters = kb_end > kb_begin ? kb_end - kb_begin : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(accum_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+    const int kchunks = static_cast<int>((args.k + 127) / 128);
+    const uint8_t* meta_tile = args.meta + row_tile * static_cast<int64_t>(kchunks) * 2048;
+    for (int i = 0; i < n_iters; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1u;
+      if (!mbar_wait(&empty_bar[s], ph ^ 1u)) { *abort_flag = 1; break; }
+      const int kb = kb_begin + i;
+      uint8_t* st = smem + s * C::kStageStride;
+      int chunks = C::kMetaChunks;
+      if (kDtype == SP24_INT8 && 2 * kb + 1 >= kchunks) chunks = 1;
+      mbar_arrive_expect_tx(&full_bar[s], C::kABytes + 2 * C::kBHalfBytes + 2048 * chunks);
+      // A: compressed columns [kb*128B) of rows [row_tile*128, +128)
+      tma_load_2d(st, &tmap_a, &full_bar[s], kb * (kDtype == SP24_BF16 ? 64 : 128),
+                  static_cast<int32_t>(row_tile * 128));
+      // B: logical K [kb*KL, +KL) of tokens [tok_tile*BN, +BN), two halves
+      const int kx = kb * C::kLogicalK;
+      const int half = C::kLogicalK / 2;
+      tma_load_2d(st + C::kABytes, &tmap_b, &full_bar[s], kx,
+                  static_cast<int32_t>(tok_tile * BN));
+      tma_load_2d(st + C::kABytes + C::kBHalfBytes, &tmap_b, &full_bar[s], kx + half,
+                  static_cast<int32_t>(tok_tile * BN));
+      // E: metadata chunk(s) of this K block
+      const int c0 = kb * C::kMetaChunks;
+      bulk_load(st + C::kABytes + 2 * C::kBHalfBytes, meta_tile + static_cast<int64_t>(c0) * 2048,
+                2048u * chunks, &full_bar[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    const int64_t k_total = args.k;
+    for (int i = 0; i < n_iters; ++i) {
+      const int s = i % STAGES;
+      const uint32_t ph = (i / STAGES) & 1u;
+      if (!mbar_wait(&full_bar[s], ph)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int kb = kb_begin + i;
+      uint8_t* st = smem + s * C::kStageStride;
+      const uint32_t a_addr = smem_u32(st);
+      const uint32_t b_addr = smem_u32(st + C::kABytes);
+      const uint32_t e_addr = smem_u32(st + C::kABytes + 2 * C::kBHalfBytes);
+      const uint32_t meta_col = C::kMetaCol0 + (i & 1) * C::kMetaCols;
+      // MMAs that touch real K positions in this stage (the tail stage may
+      // need fewer; the rest would only multiply zero fill)
+      const int64_t k_left = k_total - static_cast<int64_t>(kb) * C::kLogicalK;
+      int n_mma = static_cast<int>((k_left + C::kMmaK - 1) / C::kMmaK);
+      n_mma = n_mma > 4 ? 4 : n_mma;
+      const int chunks = kDtype == SP24_BF16 ? 1 : (n_mma > 2 ? 2 : 1);
+      for (int c = 0; c < chunks; ++c) {
+        // 128 rows x 16 bytes, rows contiguous: core matrices of 8 rows at 128 B
+        tc_cp_128x128b(tmem_base + meta_col + 4 * c,
+                       smem_desc(e_addr + 2048 * c, 128, 128, kSwizzleNone));
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j < n_mma) {
+          const uint64_t a_desc = smem_desc(a_addr + 32 * j, 0, 1024, kSwizzle128B);
+          const uint64_t b_desc =
+              smem_desc(b_addr + (j >> 1) * C::kBHalfBytes + 64 * (j & 1), 0, 1024, kSwizzle128B);
+          const uint32_t accumulate = (i > 0 || j > 0) ? 1u : 0u;
+          if constexpr (kDtype == SP24_BF16) {
+            tc_mma_sp(tmem_base, a_desc, b_desc, tmem_base + meta_col + (j & ~1),
+                      make_idesc<kDtype, BN>(j & 1), accumulate);
+          } else {
+            tc_mma_sp_i8(tmem_base, a_desc, b_desc, tmem_base + meta_col + 2 * j,
+                         make_idesc<kDtype, BN>(0), accumulate);
+          }
+        }
+      }
+      tc_commit(&empty_bar[s]);   // frees the stage once these MMAs are done
+    }
+    tc_commit(accum_bar);         // accumulator complete
+  }
+  __syncwarp();
+
+  // ---------------------------------------------------------------- epilogue
+  if (n_iters > 0 && !mbar_wait(accum_bar, 0)) *abort_flag = 1;
+  tc_fence_after();
+  __syncthreads();
+  const bool ok = *abort_flag == 0;   // uniform across the CTA
+
+  const int row_local = threadIdx.x;  // TMEM lane = output channel within the tile
+  const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+  // staging buffer reuses the (now idle) pipeline ring: [BN][128] 32-bit
+  uint32_t* stage32 = reinterpret_cast<uint32_t*>(smem);
+
+  // 1) accumulator -> shared memory, token-major (raw 32-bit accumulators)
+  if (ok && n_iters > 0) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < BN; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld16(lane_addr + c0, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) stage32[(c0 + j) * 128 + row_local] = r[j];
+    }
+  } else {
+    for (int c0 = 0; c0 < BN; ++c0) stage32[c0 * 128 + row_local] = 0u;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (SPLIT > 1) cluster_sync();   // all partials visible cluster-wide
+
+  // 2) reduce over the split CTAs (fixed rank order), scale / cast, store.
+  //    CTA `split` owns tokens [split*BN/SPLIT, (split+1)*BN/SPLIT).
+  constexpr int kTokPerCta = BN / SPLIT;
+  const int tok0 = static_cast<int>(split) * kTokPerCta;
+  // work item = (token, group of 4 channels); 32 groups per token
+  const float sx = (kDtype == SP24_INT8 && args.out_kind != SP24_OUT_INT32) ? *args.s_x : 1.0f;
+  const float sy = (kDtype == SP24_INT8 && args.out_kind == SP24_OUT_INT8) ? *args.s_y : 1.0f;
+  for (int item = threadIdx.x; item < kTokPerCta * 32; item += 128) {
+    const int t = tok0 + item / 32;
+    const int g = item % 32;
+    const int64_t m_idx = tok_tile * BN + t;
+    const int64_t n0 = row_tile * 128 + 4 * g;
+    if (m_idx >= args.m || n0 >= args.n) continue;
+    const uint32_t off = smem_u32(stage32 + t * 128 + 4 * g);
+    uint4 acc;
+    if constexpr (SPLIT > 1) {
+      acc = ld_cluster_v4(map_peer(off, 0));
+      for (int q = 1; q < SPLIT; ++q) {
+        const uint4 p = ld_cluster_v4(map_peer(off, q));
+        if constexpr (kDtype == SP24_BF16) {
+          acc.x = __float_as_uint(__fadd_rn(__uint_as_float(acc.x), __uint_as_float(p.x)));
+          acc.y = __float_as_uint(__fadd_rn(__uint_as_float(acc.y), __uint_as_float(p.y)));
+          acc.z = __float_as_uint(__fadd_rn(__uint_as_float(acc.z), __uint_as_float(p.z)));
+          acc.w = __float_as_uint(__fadd_rn(__uint_as_float(acc.w), __uint_as_float(p.w)));
+        } else {
+          acc.x += p.x; acc.y += p.y; acc.z += p.z; acc.w += p.w;
+        }
+      }
+    } else {
+      acc = *reinterpret_cast<const uint4*>(stage32 + t * 128 + 4 * g);
+    }
+    const uint32_t a4[4] = {acc.x, acc.y, acc.z, acc.w};
+    if constexpr (kDtype == SP24_BF16) {
+      __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.y) + m_idx * args.n + n0;
+      __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(a4[0]), __uint_as_float(a4[1]));
+      __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(a4[2]), __uint_as_float(a4[3]));
+      uint2 o;
+      o.x = *reinterpret_cast<uint32_t*>(&lo);
+      o.y = *reinterpret_cast<uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(y) = o;
+    } else if (args.out_kind == SP24_OUT_INT32) {
+      int32_t* y = static_cast<int32_t*>(args.y) + m_idx * args.n + n0;
+      *reinterpret_cast<uint4*>(y) = acc;
+    } else {
+      float f[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float c = __fmul_rn(sx, __ldg(args.s_w + n0 + j));
+        f[j] = __fmul_rn(__int2float_rn(static_cast<int32_t>(a4[j])), c);
+      }
+      if (args.out_kind == SP24_OUT_BF16) {
+        __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.y) + m_idx * args.n + n0;
+        __nv_bfloat162 lo = __floats2bfloat162_rn(f[0], f[1]);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(f[2], f[3]);
+        uint2 o;
+        o.x = *reinterpret_cast<uint32_t*>(&lo);
+        o.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(y) = o;
+      } else {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int q = __float2int_rn(__fdiv_rn(f[j], sy));
+          q = q > 127 ? 127 : (q < -127 ? -127 : q);
+          packed |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * j);
+        }
+        int8_t* y = static_cast<int8_t*>(args.y) + m_idx * args.n + n0;
+        *reinterpret_cast<uint32_t*>(y) = packed;
+      }
+    }
+  }
+  __syncwarp();
+  if constexpr (SPLIT > 1) cluster_sync();   // peers finished reading our partials
+
+  if (!ok) settle_ns(20000);   // let copies already in flight land
+  __syncthreads();
+  if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// ----------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2D row-major [rows][cols] map with a {box_cols, box_rows} box, 128B swizzle,
+// zero fill outside the tensor.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elsize,
+              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elsize)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kDtype, int BN, int STAGES, int SPLIT>
+sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,
+                            cudaStream_t s) {
+  using C = GemmCfg<kDtype, BN, STAGES>;
+  auto kern = gemm_sp_kernel<kDtype, BN, STAGES, SPLIT>;
+  static uint64_t attr_set = 0;   // one bit per device (devices 0..63)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SP24_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return SP24_ERR_CUDA;
+    attr_set |= bit;
+  }
+  const int64_t row_tiles = (a.n + 127) / 128;
+  const int64_t tok_tiles = (a.m + BN - 1) / BN;
+  if (row_tiles > 65535 || tok_tiles > 65535) return SP24_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(SPLIT, static_cast<unsigned>(row_tiles), static_cast<unsigned>(tok_tiles));
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = SPLIT;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return SP24_ERR_CUDA;
+  return launch_status();
+}
+
+// Tile plan: BN from the token count, split-K from how many tiles exist.
+template <int kDtype>
+sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s) {
+  const int sms = sm_count();
+  const int64_t row_tiles = (a.n + 127) / 128;
+  int bn = a.m <= 16 ? 16 : a.m <= 32 ? 32 : a.m <= 64 ? 64 : 128;
+  const int64_t tok_tiles = (a.m + bn - 1) / bn;
+  const int64_t base = row_tiles * tok_tiles;
+  int split = 1;
+  while (split < 8 && base * split < 2 * sms && a.kblocks >= 2 * split) split *= 2;
+  a.kb_per_split = (a.kblocks + split - 1) / split;
+
+  const int el = kDtype == SP24_BF16 ? 2 : 1;
+  const CUtensorMapDataType dt =
+      kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint32_t box_cols = 128 / el;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, vals, dt, el, static_cast<uint64_t>(a.k / 2), static_cast<uint64_t>(a.n),
+                box_cols, 128))
+    return SP24_ERR_CUDA;
+  if (!make_map(&mb, x, dt, el, static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.m), box_cols,
+                static_cast<uint32_t>(bn)))
+    return SP24_ERR_CUDA;
+
+#define SP24_GEMM_CASE(BN_, ST_)                                                          \
+  if (bn == BN_) {                                                                        \
+    switch (split) {                                                                      \
+      case 1: return launch_gemm_cfg<kDtype, BN_, ST_, 1>(ma, mb, a, s);                  \
+      case 2: return launch_gemm_cfg<kDtype, BN_, ST_, 2>(ma, mb, a, s);                  \
+      case 4: return launch_gemm_cfg<kDtype, BN_, ST_, 4>(ma, mb, a, s);                  \
+      default: return launch_gemm_cfg<kDtype, BN_, ST_, 8>(ma, mb, a, s);                 \
+    }                                                                                     \
+  }
+  SP24_GEMM_CASE(16, 8)
+  SP24_GEMM_CASE(32, 8)
+  SP24_GEMM_CASE(64, 6)
+  SP24_GEMM_CASE(128, 4)
+#undef SP24_GEMM_CASE
+  return SP24_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
+                                 const void* meta, int64_t N, int dtype, const float* s_x,
+                                 const float* s_w, int out_kind, const float* s_y, void* Y,
+                                 void* stream) {
+  if (M < 0 || N < 0 || K < 0 || (dtype != SP24_BF16 && dtype != SP24_INT8)) return SP24_ERR_ARG;
+  if (dtype == SP24_BF16 && out_kind != SP24_OUT_BF16) return SP24_ERR_ARG;
+  if (dtype == SP24_INT8 && out_kind != SP24_OUT_BF16 && out_kind != SP24_OUT_INT32 &&
+      out_kind != SP24_OUT_INT8)
+    return SP24_ERR_ARG;
+  if (M == 0 || N == 0) return SP24_OK;
+  if (!X || !vals || !meta || !Y) return SP24_ERR_ARG;
+  if (dtype == SP24_INT8 && out_kind != SP24_OUT_INT32 && (!s_x || !s_w)) return SP24_ERR_ARG;
+  if (dtype == SP24_INT8 && out_kind == SP24_OUT_INT8 && !s_y) return SP24_ERR_ARG;
+  if (K < 16 || N % 8 != 0 || K % (dtype == SP24_BF16 ? 16 : 32) != 0) return SP24_ERR_ALIGN;
+  if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) || !aligned16(Y) ||
+      (s_w && !aligned16(s_w)))
+    return SP24_ERR_ALIGN;
+  if (K > (int64_t(1) << 31) || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
+    return SP24_ERR_UNSUPPORTED;
+  SP24_TRY(check_device());
+  if (!get_encoder()) return SP24_ERR_CUDA;
+  GemmArgs a;
+  a.meta = static_cast<const uint8_t*>(meta);
+  a.s_x = s_x;
+  a.s_w = s_w;
+  a.s_y = s_y;
+  a.y = Y;
+  a.m = M;
+  a.n = N;
+  a.k = K;
+  a.out_kind = out_kind;
+  const int kl = dtype == SP24_BF16 ? 128 : 256;
+  a.kblocks = static_cast<int>((K + kl - 1) / kl);
+  a.kb_per_split = a.kblocks;
+  if (dtype == SP24_BF16) return dispatch<SP24_BF16>(X, vals, a, as_stream(stream));
+  return dispatch<SP24_INT8>(X, vals, a, as_stream(stream));
+}

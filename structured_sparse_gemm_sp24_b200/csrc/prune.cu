@@ -1,0 +1,619 @@
+// libsp24: Wanda column norms, N:4 pruning, compression (bf16 / int8) into the
+// tcgen05.mma.sp operand layout, INT8 calibration scales and quantisation.
+//
+// All of these are HBM-bound streaming kernels: 16-byte vector loads of W,
+// one pass over the data, grid sized in multiples of the SM count.
+//
+// Sources: [Wanda-2:4] "Structured Pruning: 2:4 sparse inference with the
+// Wanda algorithm" sections 1.3, 2.1, 2.2; [Orin ch.7] "Chapter 7: 2:4
+// Structured Sparsity" section 2.1 (worked 1x4 example: rule, compressed data
+// stream, 2-bit metadata) and 6.1 (every 1x4 block must be valid);
+// [Ampere-sparsity] NVIDIA x Tencent article, Figure 1 (values + index
+// metadata), Figure 4 (progressive 25 % -> 50 %), "PTQ and QAT" (99.99 %
+// coverage scale).
+#include "sp24_device.cuh"
+#include "sp24_host.h"
+
+namespace sp24 {
+
+// ------------------------------------------------------------- scoring keys
+// Magnitude order of a finite bf16 equals the unsigned order of its low 15
+// bits, so magnitude scores compare exactly as integers (and -0 == +0).
+__device__ __forceinline__ uint32_t mag_key(uint32_t bits16) { return bits16 & 0x7FFFu; }
+
+__device__ __forceinline__ double bf16_to_double(uint32_t bits16) {
+  return static_cast<double>(__uint_as_float(bits16 << 16));
+}
+
+// Rank rule for one group of 4: position p is kept iff fewer than n_keep
+// others beat it; for p < q, p beats q when s_p >= s_q (ties to the lower
+// index), otherwise q beats p.  Returns the keep nibble (bit p = kept).
+template <typename S>
+__device__ __forceinline__ uint32_t keep_nibble(S s0, S s1, S s2, S s3, int n_keep) {
+  int b0 = 0, b1 = 0, b2 = 0, b3 = 0;
+  if (s0 >= s1) ++b1; else ++b0;
+  if (s0 >= s2) ++b2; else ++b0;
+  if (s0 >= s3) ++b3; else ++b0;
+  if (s1 >= s2) ++b2; else ++b1;
+  if (s1 >= s3) ++b3; else ++b1;
+  if (s2 >= s3) ++b3; else ++b2;
+  return static_cast<uint32_t>(b0 < n_keep) | (static_cast<uint32_t>(b1 < n_keep) << 1) |
+         (static_cast<uint32_t>(b2 < n_keep) << 2) | (static_cast<uint32_t>(b3 < n_keep) << 3);
+}
+
+// Keep mask byte for 8 consecutive weights of one row (two groups): low
+// nibble = first group.  `w` holds the 8 bf16 patterns, `in` the mask_in byte
+// (0xFF when absent), `nrm` the 8 column norms (Wanda only).
+template <bool kWanda>
+__device__ __forceinline__ uint32_t mask_byte(const uint4& w, uint32_t in, const double* nrm,
+                                              int n_keep) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  uint32_t out = 0;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    uint32_t b[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t word = words[2 * g + i / 2];
+      const uint32_t bits = (i & 1) ? (word >> 16) : (word & 0xFFFFu);
+      const bool live = (in >> (4 * g + i)) & 1u;
+      b[i] = live ? bits : 0u;
+    }
+    uint32_t nib;
+    if constexpr (kWanda) {
+      double s[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] = __dmul_rn(fabs(bf16_to_double(b[i])), nrm[4 * g + i]);
+      nib = keep_nibble(s[0], s[1], s[2], s[3], n_keep);
+    } else {
+      nib = keep_nibble(mag_key(b[0]), mag_key(b[1]), mag_key(b[2]), mag_key(b[3]), n_keep);
+    }
+    out |= nib << (4 * g);
+  }
+  return out;
+}
+
+// -------------------------------------------------------------- a1 colnorm
+// Thread per 8 columns; sequential float64 sum over the Mc rows.
+__global__ void __launch_bounds__(256) colnorm_kernel(const uint16_t* __restrict__ xc,
+                                                      int64_t mc, int64_t k,
+                                                      double* __restrict__ norms) {
+  const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nv = k / 8;
+  if (v >= nv) return;
+  double acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
+  const uint4* p = reinterpret_cast<const uint4*>(xc) + v;
+  for (int64_t t = 0; t < mc; ++t) {
+    const uint4 q = __ldg(p + t * nv);
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t bits = (i & 1) ? (words[i / 2] >> 16) : (words[i / 2] & 0xFFFFu);
+      const double x = bf16_to_double(bits);
+      acc[i] = __dadd_rn(acc[i], __dmul_rn(x, x));  // square exact, one rounding per add
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) norms[8 * v + i] = __dsqrt_rn(acc[i]);
+}
+
+// ------------------------------------------------------------ a2+a3 prune
+// Flat over W: vector v = 8 consecutive weights = one mask byte (K % 8 == 0,
+// so a vector never straddles two rows).  Grid-stride, 4 vectors in flight.
+template <bool kWanda>
+__global__ void __launch_bounds__(256) prune_kernel(const uint4* __restrict__ w, int64_t nvec,
+                                                    int64_t kvec, const double* __restrict__ norms,
+                                                    const uint8_t* __restrict__ mask_in,
+                                                    uint8_t* __restrict__ mask_out, int n_keep) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; v < nvec; v += 4 * stride) {
+    uint4 q[4];
+    uint32_t in[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t vu = v + u * stride;
+      if (vu < nvec) {
+        q[u] = __ldcs(w + vu);
+        in[u] = mask_in ? mask_in[vu] : 0xFFu;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t vu = v + u * stride;
+      if (vu < nvec) {
+        double nrm[8];
+        if constexpr (kWanda) {
+          const int64_t col = (vu % kvec) * 8;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + col + i);
+        }
+        mask_out[vu] = static_cast<uint8_t>(mask_byte<kWanda>(q[u], in[u], nrm, n_keep));
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ a4 compress
+// Metadata operand layout (per 128-row x 128-K chunk, 2048 bytes; chunks
+// ordered [row tile][K block]).  Source byte = (row m, byte bb of the chunk's
+// 16 metadata bytes per row), covering groups 2bb, 2bb+1 of the chunk.
+//   int8 (tcgen05 kind::i8): row-major, offset = 16*m + bb.
+//   bf16 (kind::f16): tensor-memory lane = (m%8) + 8*((bb%4)/2) + 16*(m/16);
+//        within the lane, 32-bit word j = bb/4 feeds MMA j (32 K-positions);
+//        rows m%16 < 8 fill the low half-word and rows m%16 >= 8 the high one;
+//        offset = 16*lane + 4*j + 2*((m/8)%2) + (bb%2).
+// Nibble order inside a byte is the same as in the canonical layout.
+template <int kDtype>
+__device__ __forceinline__ uint32_t meta_offset(uint32_t m, uint32_t bb) {
+  if constexpr (kDtype == SP24_INT8) {
+    return 16u * m + bb;
+  } else {
+    const uint32_t lane = (m & 7u) + 8u * ((bb & 3u) >> 1) + 16u * (m >> 4);
+    return 16u * lane + 4u * (bb >> 2) + 2u * ((m >> 3) & 1u) + (bb & 1u);
+  }
+}
+
+// Kept positions of a nibble with exactly two bits set -> (lo | hi << 2).
+// Any other nibble is a pattern error; it is recorded and encoded as (0, 1).
+__device__ __forceinline__ uint32_t meta_nibble(uint32_t keep, uint32_t& bad) {
+  const uint32_t lo = __ffs(keep) - 1u;
+  const uint32_t hi = 31u - __clz(keep);
+  const bool ok = __popc(keep) == 2;
+  bad |= ok ? 0u : 1u;
+  return ok ? (lo | (hi << 2)) : 0x4u;
+}
+
+template <int kDtype>
+struct CompressOut;
+
+// One CTA per metadata chunk (128 rows x 128 K).  256 threads, each takes one
+// 8-weight vector per step (16 vectors per chunk row), so a warp reads two
+// chunk rows of 256 contiguous bytes.  The metadata chunk is assembled in
+// shared memory and written out with 16-byte stores.
+//
+// kPrune: compute the keep mask here (magnitude / Wanda, n_keep = 2) instead
+// of reading it; optionally also write it to mask_out.
+template <int kDtype, bool kPrune, bool kWanda>
+__global__ void __launch_bounds__(256)
+compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask,
+                const uint8_t* __restrict__ mask_in, uint8_t* __restrict__ mask_out,
+                const double* __restrict__ norms, const float* __restrict__ s_w, int64_t n,
+                int64_t k, void* __restrict__ vals, uint8_t* __restrict__ meta) {
+  __shared__ __align__(16) uint8_t chunk[2048];
+  const int64_t kb = blockIdx.x;                 // K block of 128
+  const int64_t rt = blockIdx.y;                 // row tile of 128
+  const int64_t kblocks = gridDim.x;
+  const int64_t kvec = k / 8;
+  uint32_t bad = 0;
+
+  for (int step = 0; step < 8; ++step) {
+    const uint32_t idx = step * 256u + threadIdx.x;   // 0 .. 2047
+    const uint32_t m = idx >> 4;                      // chunk row
+    const uint32_t bb = idx & 15u;                    // vector within the chunk row
+    const int64_t row = rt * 128 + m;
+    const int64_t kv = kb * 16 + bb;                  // vector index within the row
+    uint32_t meta_byte = 0x44u;                       // padding: positions (0,1)
+    if (row < n && kv < kvec) {
+      const int64_t vi = row * kvec + kv;
+      const uint4 q = __ldcs(reinterpret_cast<const uint4*>(w) + vi);
+      uint32_t keep;
+      if constexpr (kPrune) {
+        double nrm[8];
+        if constexpr (kWanda) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + kv * 8 + i);
+        }
+        keep = mask_byte<kWanda>(q, mask_in ? mask_in[vi] : 0xFFu, nrm, 2);
+        if (mask_out) mask_out[vi] = static_cast<uint8_t>(keep);
+      } else {
+        keep = mask[vi];
+      }
+      const uint32_t n0 = meta_nibble(keep & 15u, bad);
+      const uint32_t n1 = meta_nibble(keep >> 4, bad);
+      meta_byte = n0 | (n1 << 4);
+      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+      uint32_t sel[4];
+      const uint32_t pos[4] = {n0 & 3u, n0 >> 2, 4u + (n1 & 3u), 4u + (n1 >> 2)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t word = words[pos[i] >> 1];
+        sel[i] = (pos[i] & 1u) ? (word >> 16) : (word & 0xFFFFu);
+      }
+      if constexpr (kDtype == SP24_BF16) {
+        uint2 o;
+        o.x = sel[0] | (sel[1] << 16);
+        o.y = sel[2] | (sel[3] << 16);
+        reinterpret_cast<uint2*>(vals)[vi] = o;
+      } else {
+        const float s = s_w[row];
+        uint32_t packed = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float x = __uint_as_float(sel[i] << 16);
+          int qv = __float2int_rn(__fdiv_rn(x, s));
+          qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
+          packed |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * i);
+        }
+        reinterpret_cast<uint32_t*>(vals)[vi] = packed;
+      }
+    }
+    chunk[meta_offset<kDtype>(m, bb)] = static_cast<uint8_t>(meta_byte);
+  }
+  if (bad) raise_error(kErrPatternBit);
+  __syncthreads();
+  if (threadIdx.x < 128) {
+    uint4* dst = reinterpret_cast<uint4*>(meta + (rt * kblocks + kb) * 2048);
+    dst[threadIdx.x] = reinterpret_cast<const uint4*>(chunk)[threadIdx.x];
+  }
+}
+
+// --------------------------------------------------------- a5 weight scale
+// One CTA per row.  Keys = |w| bit patterns (15 bits) of the kept positions;
+// the r-th smallest key is found with two histogram passes (high 8 bits, then
+// low 7 bits within the selected bucket).
+__global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict__ w,
+                                                     const uint8_t* __restrict__ mask,
+                                                     int64_t k, double coverage,
+                                                     float* __restrict__ s_w) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t s_count, s_bucket, s_rank;
+  const int64_t row = blockIdx.x;
+  const uint16_t* wr = w + row * k;
+  const uint8_t* mr = mask + row * (k / 8);
+  const int64_t kvec = k / 8;
+
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+  if (threadIdx.x == 0) s_count = 0;
+  __syncthreads();
+  uint32_t cnt = 0;
+  for (int64_t v = threadIdx.x; v < kvec; v += blockDim.x) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
+    const uint32_t keep = mr[v];
+    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((keep >> i) & 1u) {
+        const uint32_t key = mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]);
+        atomicAdd(&hist[key >> 7], 1u);
+        ++cnt;
+      }
+    }
+  }
+  atomicAdd(&s_count, cnt);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t c = s_count;
+    uint32_t r = c == 0 ? 0u : static_cast<uint32_t>(ceil(coverage * static_cast<double>(c)));
+    if (r < 1) r = 1;
+    if (r > c) r = c;
+    uint32_t below = 0, b = 0;
+    for (b = 0; b < 256; ++b) {
+      if (below + hist[b] >= r) break;
+      below += hist[b];
+    }
+    s_bucket = b;
+    s_rank = r - below;  // rank within the bucket, 1-based
+  }
+  __syncthreads();
+  const uint32_t c = s_count;
+  const uint32_t bucket = s_bucket;
+  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  if (c > 0) {
+    for (int64_t v = threadIdx.x; v < kvec; v += blockDim.x) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
+      const uint32_t keep = mr[v];
+      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if ((keep >> i) & 1u) {
+          const uint32_t key = mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]);
+          if ((key >> 7) == bucket) atomicAdd(&hist[key & 0x7Fu], 1u);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 1.0f;
+    if (c > 0) {
+      uint32_t below = 0, b = 0;
+      for (b = 0; b < 128; ++b) {
+        if (below + hist[b] >= s_rank) break;
+        below += hist[b];
+      }
+      const uint32_t key = (bucket << 7) | b;
+      const float t = __uint_as_float(key << 16);
+      if (t != 0.0f) s = __fdiv_rn(t, 127.0f);
+    }
+    s_w[row] = s;
+  }
+}
+
+// ----------------------------------------------------- a5 activation scale
+// Exact radix selection of the r-th smallest |x| over a float32 tensor:
+// keys = bits & 0x7FFFFFFF (monotone in |x| for finite x), three passes of
+// 11/11/9 bits.  Workspace: 2048 histogram counters + {prefix, rank}.
+struct ActScaleWs {
+  uint32_t hist[2048];
+  uint32_t prefix;   // selected high bits so far
+  uint32_t rank;     // remaining 1-based rank within the current prefix
+  uint32_t pad[2];
+};
+
+__global__ void act_scale_init(ActScaleWs* ws, uint32_t rank) {
+  for (int i = threadIdx.x; i < 2048; i += blockDim.x) ws->hist[i] = 0;
+  if (threadIdx.x == 0) {
+    ws->prefix = 0;
+    ws->rank = rank;
+  }
+}
+
+__global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__ x, int64_t nvec,
+                                                      const float* __restrict__ tail,
+                                                      int ntail, ActScaleWs* ws, int shift,
+                                                      int bits, uint32_t hi_mask) {
+  __shared__ uint32_t h[2048];
+  const uint32_t nb = 1u << bits;
+  for (uint32_t i = threadIdx.x; i < nb; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const uint32_t prefix = ws->prefix;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec;
+       v += stride) {
+    const float4 q = __ldcs(x + v);
+    const float e[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t key = __float_as_uint(e[i]) & 0x7FFFFFFFu;
+      if ((key & hi_mask) == prefix) atomicAdd(&h[(key >> shift) & (nb - 1u)], 1u);
+    }
+  }
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < ntail; i += blockDim.x) {
+      const uint32_t key = __float_as_uint(tail[i]) & 0x7FFFFFFFu;
+      if ((key & hi_mask) == prefix) atomicAdd(&h[(key >> shift) & (nb - 1u)], 1u);
+    }
+  }
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < nb; i += blockDim.x)
+    if (h[i]) atomicAdd(&ws->hist[i], h[i]);
+}
+
+__global__ void act_scale_select(ActScaleWs* ws, int shift, int bits, float* s_x, int last) {
+  if (threadIdx.x != 0) return;
+  const uint32_t nb = 1u << bits;
+  uint32_t below = 0, b = 0;
+  for (b = 0; b < nb - 1u; ++b) {
+    if (below + ws->hist[b] >= ws->rank) break;
+    below += ws->hist[b];
+  }
+  ws->prefix |= b << shift;
+  ws->rank -= below;
+  for (uint32_t i = 0; i < nb; ++i) ws->hist[i] = 0;
+  if (last) {
+    const float t = __uint_as_float(ws->prefix);
+    *s_x = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
+  }
+}
+
+// ----------------------------------------------------------- quantisation
+__device__ __forceinline__ uint32_t q8(float x, float s) {
+  int q = __float2int_rn(__fdiv_rn(x, s));
+  q = q > 127 ? 127 : (q < -127 ? -127 : q);
+  return static_cast<uint32_t>(q) & 0xFFu;
+}
+
+__global__ void __launch_bounds__(256) quantize_kernel(const float4* __restrict__ x, int64_t nvec16,
+                                                       const float* __restrict__ s_ptr,
+                                                       uint4* __restrict__ xq) {
+  const float s = *s_ptr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec16;
+       v += stride) {
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 q = __ldcs(x + 4 * v + j);
+      out[j] = q8(q.x, s) | (q8(q.y, s) << 8) | (q8(q.z, s) << 16) | (q8(q.w, s) << 24);
+    }
+    xq[v] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+__global__ void quantize_tail(const float* __restrict__ x, int64_t start, int64_t count,
+                              const float* __restrict__ s_ptr, int8_t* __restrict__ xq) {
+  const int64_t i = start + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < count) xq[i] = static_cast<int8_t>(q8(x[i], *s_ptr));
+}
+
+// -------------------------------------------------------------- launching
+static int grid_for(int64_t work_items, int threads) {
+  const int64_t want = (work_items + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
+  return static_cast<int>(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double* norms,
+                                  cudaStream_t s) {
+  const int64_t nv = k / 8;
+  const int blocks = static_cast<int>((nv + 255) / 256);
+  colnorm_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(xc), mc, k, norms);
+  return launch_status();
+}
+
+template <int kDtype, bool kPrune, bool kWanda>
+static sp24_status launch_compress(const void* w, const uint8_t* mask, const uint8_t* mask_in,
+                                   uint8_t* mask_out, const double* norms, const float* s_w,
+                                   int64_t n, int64_t k, void* vals, void* meta, cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>((k + 127) / 128), static_cast<unsigned>((n + 127) / 128));
+  compress_kernel<kDtype, kPrune, kWanda><<<grid, 256, 0, s>>>(
+      static_cast<const uint16_t*>(w), mask, mask_in, mask_out, norms, s_w, n, k, vals,
+      static_cast<uint8_t*>(meta));
+  return launch_status();
+}
+
+}  // namespace sp24
+
+using namespace sp24;
+
+extern "C" {
+
+sp24_status sp24_colnorm(const void* Xc, int64_t Mc, int64_t K, double* norms, void* stream) {
+  if (!Xc || !norms || Mc < 1 || K < 1) return SP24_ERR_ARG;
+  if (K % 8 != 0 || !aligned16(Xc) || !aligned16(norms)) return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  return launch_colnorm(Xc, Mc, K, norms, as_stream(stream));
+}
+
+sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc, int64_t Mc,
+                       int mode, int n_keep, const uint8_t* mask_in, uint8_t* mask_out,
+                       void* workspace, void* stream) {
+  if (N < 0 || K < 0 || (mode != SP24_MAGNITUDE && mode != SP24_WANDA) ||
+      (n_keep != 2 && n_keep != 3))
+    return SP24_ERR_ARG;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!W || !mask_out) return SP24_ERR_ARG;
+  if (mode == SP24_WANDA && (!Xc || Mc < 1 || !workspace)) return SP24_ERR_ARG;
+  if (K % 8 != 0 || !aligned16(W) || !aligned16(mask_out) || (mask_in && !aligned16(mask_in)))
+    return SP24_ERR_ALIGN;
+  if (mode == SP24_WANDA && (!aligned16(Xc) || !aligned16(workspace))) return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  const int64_t nvec = N * (K / 8);
+  const int grid = grid_for((nvec + 3) / 4, 256);
+  if (mode == SP24_WANDA) {
+    double* norms = static_cast<double*>(workspace);
+    SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
+    prune_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W), nvec, K / 8, norms,
+                                            mask_in, mask_out, n_keep);
+  } else {
+    prune_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W), nvec, K / 8, nullptr,
+                                             mask_in, mask_out, n_keep);
+  }
+  return launch_status();
+}
+
+sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K,
+                        double coverage, float* s_w, void* stream) {
+  if (N < 0 || K < 0 || !(coverage > 0.0 && coverage <= 1.0)) return SP24_ERR_ARG;
+  if (N == 0) return SP24_OK;
+  if (!W || !mask || !s_w) return SP24_ERR_ARG;
+  if (K % 8 != 0 || !aligned16(W) || !aligned16(mask) || !aligned16(s_w)) return SP24_ERR_ALIGN;
+  if (N > 0x7FFFFFFF) return SP24_ERR_ARG;
+  SP24_TRY(check_device());
+  wscale_kernel<<<static_cast<unsigned>(N), 256, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(W), mask, K, coverage, s_w);
+  return launch_status();
+}
+
+size_t sp24_act_scale_workspace_bytes(void) { return sizeof(ActScaleWs); }
+
+sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float* s_x,
+                           void* workspace, void* stream) {
+  if (!X || !s_x || !workspace || count < 1 || !(coverage > 0.0 && coverage <= 1.0))
+    return SP24_ERR_ARG;
+  if (count > 0x7FFFFFFFll) return SP24_ERR_ARG;
+  if (!aligned16(X) || !aligned16(workspace)) return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  double rd = ceil(coverage * static_cast<double>(count));
+  uint32_t rank = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
+  if (rank > static_cast<uint64_t>(count)) rank = static_cast<uint32_t>(count);
+  ActScaleWs* ws = static_cast<ActScaleWs*>(workspace);
+  act_scale_init<<<1, 256, 0, s>>>(ws, rank);
+  SP24_TRY(launch_status());
+  const int64_t nvec = count / 4;
+  const int ntail = static_cast<int>(count - nvec * 4);
+  const int grid = grid_for(nvec, 256);
+  const int shifts[3] = {20, 9, 0};
+  const int bitsv[3] = {11, 11, 9};
+  uint32_t hi_mask = 0;
+  for (int p = 0; p < 3; ++p) {
+    act_scale_hist<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(X), nvec,
+                                        X + nvec * 4, ntail, ws, shifts[p], bitsv[p], hi_mask);
+    SP24_TRY(launch_status());
+    act_scale_select<<<1, 32, 0, s>>>(ws, shifts[p], bitsv[p], s_x, p == 2);
+    SP24_TRY(launch_status());
+    hi_mask |= ((1u << bitsv[p]) - 1u) << shifts[p];
+  }
+  return SP24_OK;
+}
+
+sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x, int8_t* Xq,
+                          void* stream) {
+  if (count < 0) return SP24_ERR_ARG;
+  if (count == 0) return SP24_OK;
+  if (!X || !s_x || !Xq) return SP24_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Xq)) return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  const int64_t nvec16 = count / 16;
+  if (nvec16 > 0) {
+    quantize_kernel<<<grid_for(nvec16, 256), 256, 0, s>>>(reinterpret_cast<const float4*>(X),
+                                                         nvec16, s_x,
+                                                         reinterpret_cast<uint4*>(Xq));
+    SP24_TRY(launch_status());
+  }
+  const int64_t start = nvec16 * 16;
+  if (start < count) {
+    quantize_tail<<<1, 32, 0, s>>>(X, start, count, s_x, Xq);
+    SP24_TRY(launch_status());
+  }
+  return SP24_OK;
+}
+
+sp24_status sp24_compress(const void* W, const uint8_t* mask, int64_t N, int64_t K, int dtype,
+                          const float* s_w, void* vals, void* meta, void* stream) {
+  if (N < 0 || K < 0 || (dtype != SP24_BF16 && dtype != SP24_INT8)) return SP24_ERR_ARG;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!W || !mask || !vals || !meta || (dtype == SP24_INT8 && !s_w)) return SP24_ERR_ARG;
+  if (K % (dtype == SP24_BF16 ? 16 : 32) != 0) return SP24_ERR_ALIGN;
+  if (!aligned16(W) || !aligned16(mask) || !aligned16(vals) || !aligned16(meta) ||
+      (s_w && !aligned16(s_w)))
+    return SP24_ERR_ALIGN;
+  if ((N + 127) / 128 > 65535) return SP24_ERR_ARG;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  if (dtype == SP24_BF16)
+    return launch_compress<SP24_BF16, false, false>(W, mask, nullptr, nullptr, nullptr, nullptr, N,
+                                                     K, vals, meta, s);
+  return launch_compress<SP24_INT8, false, false>(W, mask, nullptr, nullptr, nullptr, s_w, N, K,
+                                                  vals, meta, s);
+}
+
+sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
+                                const double* norms, const uint8_t* mask_in, uint8_t* mask_out,
+                                int dtype, const float* s_w, void* vals, void* meta,
+                                void* stream) {
+  if (N < 0 || K < 0 || (dtype != SP24_BF16 && dtype != SP24_INT8) ||
+      (mode != SP24_MAGNITUDE && mode != SP24_WANDA))
+    return SP24_ERR_ARG;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!W || !vals || !meta || (dtype == SP24_INT8 && !s_w) || (mode == SP24_WANDA && !norms))
+    return SP24_ERR_ARG;
+  if (K % (dtype == SP24_BF16 ? 16 : 32) != 0) return SP24_ERR_ALIGN;
+  if (!aligned16(W) || !aligned16(vals) || !aligned16(meta) || (s_w && !aligned16(s_w)) ||
+      (mask_in && !aligned16(mask_in)) || (mask_out && !aligned16(mask_out)) ||
+      (norms && !aligned16(norms)))
+    return SP24_ERR_ALIGN;
+  if ((N + 127) / 128 > 65535) return SP24_ERR_ARG;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  const bool wanda = mode == SP24_WANDA;
+  if (dtype == SP24_BF16) {
+    return wanda ? launch_compress<SP24_BF16, true, true>(W, nullptr, mask_in, mask_out, norms,
+                                                           nullptr, N, K, vals, meta, s)
+                 : launch_compress<SP24_BF16, true, false>(W, nullptr, mask_in, mask_out,
+                                                            nullptr, nullptr, N, K, vals, meta, s);
+  }
+  return wanda ? launch_compress<SP24_INT8, true, true>(W, nullptr, mask_in, mask_out, norms, s_w,
+                                                         N, K, vals, meta, s)
+               : launch_compress<SP24_INT8, true, false>(W, nullptr, mask_in, mask_out, nullptr,
+                                                          s_w, N, K, vals, meta, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,35 @@
+// Host-side helpers shared by the libsp24 translation units: argument
+// checks, CUDA error mapping and the sm_100 device check.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sp24.h"
+
+namespace sp24 {
+
+inline bool aligned16(const void* p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// SP24_OK when the current device is an sm_100 part (cached per device).
+sp24_status check_device();
+
+// Maps the launch status of the last kernel to a library status.
+inline sp24_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+}
+
+// Number of SMs of the current device (cached).
+int sm_count();
+
+}  // namespace sp24
+
+#define SP24_TRY(expr)                    \
+  do {                                    \
+    sp24_status _st = (expr);             \
+    if (_st != SP24_OK) return _st;       \
+  } while (0)

@@ -1,0 +1,98 @@
+"""Allocate-and-call helpers over the libsp24 binding.
+
+torch provides the device memory and the current stream; every step runs in
+the library's kernels through :mod:`structured_sparse_gemm_sp24_b200.sp24`.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import sp24 as _b
+
+COVERAGE = 0.9999   # "scale covering 99.99 % of the values" (PTQ calibration)
+
+
+def _u8(nbytes: int, device) -> torch.Tensor:
+    # 16 extra bytes keep zero-size requests valid; torch allocations are
+    # 256-byte aligned.
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def colnorm(Xc: torch.Tensor) -> torch.Tensor:
+    norms = torch.empty(Xc.shape[1], dtype=torch.float64, device=Xc.device)
+    _b.sp24_colnorm(Xc, norms)
+    return norms
+
+
+def prune(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE, n_keep: int = 2,
+          Xc: Optional[torch.Tensor] = None, mask_in: Optional[torch.Tensor] = None,
+          workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Keep mask uint8 [N, K/8] (nibble per group, bit p = position p kept)."""
+    N, K = W.shape
+    mask = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    if mode == _b.SP24_WANDA and workspace is None:
+        workspace = _u8(_b.sp24_prune_workspace_bytes(K, mode), W.device)
+    _b.sp24_prune(W, Xc, mode, n_keep, mask_in, mask, workspace)
+    return mask
+
+
+def wscale(W: torch.Tensor, mask: torch.Tensor, coverage: float = COVERAGE) -> torch.Tensor:
+    s_w = torch.empty(W.shape[0], dtype=torch.float32, device=W.device)
+    _b.sp24_wscale(W, mask, coverage, s_w)
+    return s_w
+
+
+def act_scale(X: torch.Tensor, coverage: float = COVERAGE,
+              workspace: Optional[torch.Tensor] = None) -> torch.Tensor:
+    s_x = torch.empty(4, dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = _u8(_b.sp24_act_scale_workspace_bytes(), X.device)
+    _b.sp24_act_scale(X, coverage, s_x, workspace)
+    return s_x[:1]
+
+
+def quantize(X: torch.Tensor, s_x: torch.Tensor) -> torch.Tensor:
+    Xq = torch.empty(X.shape, dtype=torch.int8, device=X.device)
+    _b.sp24_quantize(X, s_x, Xq)
+    return Xq
+
+
+def alloc_compressed(N: int, K: int, dtype: int, device) -> Tuple[torch.Tensor, torch.Tensor]:
+    tdt = torch.bfloat16 if dtype == _b.SP24_BF16 else torch.int8
+    vals = torch.empty((N, K // 2), dtype=tdt, device=device)
+    meta = _u8(_b.sp24_meta_bytes(N, K), device)
+    return vals, meta
+
+
+def compress(W: torch.Tensor, mask: torch.Tensor, dtype: int = _b.SP24_BF16,
+             s_w: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    N, K = W.shape
+    vals, meta = alloc_compressed(N, K, dtype, W.device)
+    _b.sp24_compress(W, mask, dtype, s_w, vals, meta)
+    return vals, meta
+
+
+def prune_compress(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE,
+                   norms: Optional[torch.Tensor] = None, mask_in: Optional[torch.Tensor] = None,
+                   dtype: int = _b.SP24_BF16, s_w: Optional[torch.Tensor] = None,
+                   want_mask: bool = False):
+    N, K = W.shape
+    vals, meta = alloc_compressed(N, K, dtype, W.device)
+    mask = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device) if want_mask else None
+    _b.sp24_prune_compress(W, mode, norms, mask_in, mask, dtype, s_w, vals, meta)
+    return (vals, meta, mask) if want_mask else (vals, meta)
+
+
+def gemm(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, N: int,
+         dtype: int = _b.SP24_BF16, s_x: Optional[torch.Tensor] = None,
+         s_w: Optional[torch.Tensor] = None, out_kind: int = _b.SP24_OUT_BF16,
+         s_y: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    M = X.shape[0]
+    if out is None:
+        odt = {_b.SP24_OUT_BF16: torch.bfloat16, _b.SP24_OUT_INT32: torch.int32,
+               _b.SP24_OUT_INT8: torch.int8}[out_kind]
+        out = torch.empty((M, N), dtype=odt, device=X.device)
+    _b.sp24_gemm(X, vals, meta, N, dtype, s_x, s_w, out_kind, s_y, out)
+    return out

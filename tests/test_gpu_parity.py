@@ -1,0 +1,401 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Bars: masks, metadata, int8 values, int32 accumulators, dequantised bf16 and
+requantised int8 outputs are bit-exact; the bf16 GEMM satisfies, per element,
+|y_gpu - y_ref| <= 8e-3 * sum_k |x_k * w_k| (y_ref and the bound in float64).
+Inputs are the seeded workloads of structured_sparse_gemm_sp24_b200.inputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import sp24_oracle as O
+from structured_sparse_gemm_sp24_b200 import inputs as I
+from structured_sparse_gemm_sp24_b200 import pipeline as P
+from structured_sparse_gemm_sp24_b200 import sp24 as B
+from tests import meta_layout as L
+
+pytestmark = pytest.mark.gpu
+
+TOL = 8e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _device():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    torch.cuda.set_device(0)
+    B.lib()
+    assert B.sp24_device_status() == B.SP24_OK
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def keep_of(mask_dev: torch.Tensor, k: int) -> np.ndarray:
+    return O.unpack_mask(mask_dev.cpu().numpy(), k)
+
+
+def canon_meta(meta_dev, n, k, dtype):
+    return L.decode(meta_dev.cpu().numpy(), n, k, dtype)
+
+
+def assert_bf16_close(y_dev, y_ref, a_ref):
+    y = f64(y_dev)
+    d = np.abs(y - y_ref)
+    ok = d <= TOL * a_ref
+    if not ok.all():
+        i = np.argwhere(~ok)[0]
+        raise AssertionError(
+            f"bf16 GEMM off at {tuple(i)}: gpu={y[tuple(i)]} ref={y_ref[tuple(i)]} "
+            f"bound={TOL * a_ref[tuple(i)]} ({(~ok).sum()} of {ok.size} elements)")
+    return float((d / np.where(a_ref > 0, a_ref, 1)).max())
+
+
+def ok_status():
+    assert B.sp24_device_status() == B.SP24_OK
+
+
+# ------------------------------------------------------------------ a1
+def test_colnorm_bert_calibration():
+    w = I.bert_fc1()
+    n = P.colnorm(w.Xc.cuda())
+    assert np.array_equal(n.cpu().numpy(), O.column_norms(f64(w.Xc)))
+    ok_status()
+
+
+def test_colnorm_sums_in_token_order():
+    xc = torch.zeros((33, 16), dtype=torch.bfloat16)
+    xc[:32, 0] = 2.0 ** -27
+    xc[32, 0] = 1.0
+    xc[0, 8] = 1.0
+    xc[1:, 8] = 2.0 ** -27
+    n = P.colnorm(xc.cuda()).cpu().numpy()
+    assert n[0] == 1.0 + 2.0 ** -50 and n[8] == 1.0
+    assert np.array_equal(n, O.column_norms(f64(xc)))
+
+
+# ------------------------------------------------------------------ a2/a3
+PRUNE_SHAPES = [(64, 128, 1.0), (3072, 768, 0.02), (200, 136, 0.02), (1, 8, 1.0), (130, 264, 1.0)]
+
+
+@pytest.mark.parametrize("n_keep", [2, 3])
+@pytest.mark.parametrize("shape", PRUNE_SHAPES)
+def test_prune_magnitude(shape, n_keep):
+    n, k, sigma = shape
+    w = I.normal_bf16((n, k), sigma, seed=11)
+    mask = P.prune(w.cuda(), B.SP24_MAGNITUDE, n_keep)
+    assert np.array_equal(keep_of(mask, k), O.prune(f64(w), O.MAGNITUDE, n_keep))
+    ok_status()
+
+
+def test_prune_ties_heavy():
+    # a 5-value alphabet makes ties common; -0.0 and +0.0 both appear
+    g = torch.Generator().manual_seed(5)
+    w = (torch.randint(-2, 3, (257, 512), generator=g).float() * 0.5).to(torch.bfloat16)
+    w[0, :4] = torch.tensor([0.0, -0.0, 0.0, -0.0])
+    for n_keep in (2, 3):
+        mask = P.prune(w.cuda(), B.SP24_MAGNITUDE, n_keep)
+        assert np.array_equal(keep_of(mask, 512), O.prune(f64(w), O.MAGNITUDE, n_keep))
+
+
+@pytest.mark.parametrize("n_keep", [2, 3])
+def test_prune_wanda_bert(n_keep):
+    w = I.bert_fc1()
+    mask = P.prune(w.W.cuda(), B.SP24_WANDA, n_keep, Xc=w.Xc.cuda())
+    ref = O.prune(f64(w.W), O.WANDA, n_keep, xc=f64(w.Xc))
+    assert np.array_equal(keep_of(mask, w.K), ref)
+
+
+def test_progressive_bert():
+    w = I.bert_fc1()
+    Wd, Xc = w.W.cuda(), w.Xc.cuda()
+    m1 = P.prune(Wd, B.SP24_WANDA, 3, Xc=Xc)
+    m2 = P.prune(Wd, B.SP24_WANDA, 2, Xc=Xc, mask_in=m1)
+    r1, r2 = O.progressive(f64(w.W), O.WANDA, f64(w.Xc))
+    assert np.array_equal(keep_of(m1, w.K), r1)
+    assert np.array_equal(keep_of(m2, w.K), r2)
+
+
+def test_prune_llm_full():
+    w = I.llm_proj(11008, 4096, 16)
+    mask = P.prune(w.W.cuda(), B.SP24_MAGNITUDE, 2)
+    assert np.array_equal(keep_of(mask, 4096), O.prune(f64(w.W), O.MAGNITUDE, 2))
+
+
+# ------------------------------------------------------------------ a4
+COMPRESS_SHAPES = [(64, 128), (200, 160), (3072, 768), (8, 32), (129, 288)]
+
+
+@pytest.mark.parametrize("shape", COMPRESS_SHAPES)
+def test_compress_bf16(shape):
+    n, k = shape
+    w = I.normal_bf16((n, k), 1.0, seed=3)
+    wd = w.cuda()
+    mask = P.prune(wd, B.SP24_MAGNITUDE, 2)
+    vals, meta = P.compress(wd, mask, B.SP24_BF16)
+    keep = O.prune(f64(w), O.MAGNITUDE, 2)
+    rv, rm = O.compress(f64(w), keep)
+    assert np.array_equal(f64(vals), rv)
+    assert np.array_equal(canon_meta(meta, n, k, L.BF16), rm)
+    assert L.padding_is_valid(meta.cpu().numpy(), n, k, L.BF16)
+    ok_status()
+
+
+@pytest.mark.parametrize("shape", COMPRESS_SHAPES)
+def test_compress_int8(shape):
+    n, k = shape
+    w = I.long_tail_bf16((n, k), 0.02, seed=4, tail_seed=7)
+    wd = w.cuda()
+    mask = P.prune(wd, B.SP24_MAGNITUDE, 2)
+    s_w = P.wscale(wd, mask)
+    vals, meta = P.compress(wd, mask, B.SP24_INT8, s_w)
+    keep = O.prune(f64(w), O.MAGNITUDE, 2)
+    rs = O.channel_scales(f64(w), keep)
+    assert np.array_equal(s_w.cpu().numpy(), rs)
+    wq = O.quantize(f64(w), rs[:, None])
+    rv, rm = O.compress(wq, keep)
+    assert np.array_equal(vals.cpu().numpy(), rv)
+    assert np.array_equal(canon_meta(meta, n, k, L.INT8), rm)
+    assert L.padding_is_valid(meta.cpu().numpy(), n, k, L.INT8)
+    ok_status()
+
+
+@pytest.mark.parametrize("dtype", [B.SP24_BF16, B.SP24_INT8])
+@pytest.mark.parametrize("mode", [B.SP24_MAGNITUDE, B.SP24_WANDA])
+def test_prune_compress_fused(mode, dtype):
+    w = I.bert_fc1()
+    Wd, Xc = w.W.cuda(), w.Xc.cuda()
+    m1 = P.prune(Wd, mode, 3, Xc=Xc)
+    norms = P.colnorm(Xc) if mode == B.SP24_WANDA else None
+    s_w = None
+    if dtype == B.SP24_INT8:
+        s_w = P.wscale(Wd, P.prune(Wd, mode, 2, Xc=Xc, mask_in=m1))
+    vals, meta, mask = P.prune_compress(Wd, mode, norms, m1, dtype, s_w, want_mask=True)
+    omode = O.WANDA if mode == B.SP24_WANDA else O.MAGNITUDE
+    r1 = O.prune(f64(w.W), omode, 3, xc=f64(w.Xc))
+    keep = O.prune(f64(w.W), omode, 2, xc=f64(w.Xc), mask_in=r1)
+    assert np.array_equal(keep_of(mask, w.K), keep)
+    if dtype == B.SP24_BF16:
+        rv, rm = O.compress(f64(w.W), keep)
+        assert np.array_equal(f64(vals), rv)
+    else:
+        rs = O.channel_scales(f64(w.W), keep)
+        rv, rm = O.compress(O.quantize(f64(w.W), rs[:, None]), keep)
+        assert np.array_equal(vals.cpu().numpy(), rv)
+    ldt = L.BF16 if dtype == B.SP24_BF16 else L.INT8
+    assert np.array_equal(canon_meta(meta, w.N, w.K, ldt), rm)
+    ok_status()
+
+
+def test_compress_rejects_bad_pattern():
+    w = I.normal_bf16((64, 128), 1.0, seed=1).cuda()
+    mask = P.prune(w, B.SP24_MAGNITUDE, 2)
+    ok_status()
+    bad = mask.clone()
+    bad[5, 3] = 0x7F          # groups keeping 3 and 4 positions
+    P.compress(w, bad, B.SP24_BF16)
+    assert B.sp24_device_status() == B.SP24_ERR_PATTERN
+    ok_status()               # reading the status cleared it
+    m3 = P.prune(w, B.SP24_MAGNITUDE, 3)
+    P.compress(w, m3, B.SP24_BF16)
+    assert B.sp24_device_status() == B.SP24_ERR_PATTERN
+
+
+# ------------------------------------------------------------------ a5
+def test_wscale_long_tail_full():
+    w = I.int8_long_tail()
+    wd = w.W.cuda()
+    mask = P.prune(wd, B.SP24_MAGNITUDE, 2)
+    keep = keep_of(mask, w.K)
+    assert np.array_equal(P.wscale(wd, mask).cpu().numpy(), O.channel_scales(f64(w.W), keep))
+
+
+@pytest.mark.parametrize("coverage", [0.9, 0.5, 1.0, 1e-9])
+def test_wscale_ranks_below_max(coverage):
+    w = I.normal_bf16((300, 4096), 0.02, seed=9)
+    w[7] = 0.0                                   # zero row -> scale 1
+    wd = w.cuda()
+    for n_keep in (2, 3):
+        mask = P.prune(wd, B.SP24_MAGNITUDE, n_keep)
+        got = P.wscale(wd, mask, coverage).cpu().numpy()
+        ref = O.channel_scales(f64(w), keep_of(mask, 4096), coverage)
+        assert np.array_equal(got, ref)
+        assert got[7] == 1.0
+
+
+@pytest.mark.parametrize("count", [1, 17, 4096, 1000003])
+def test_act_scale_and_quantize_small(count):
+    x = I.normal_f32((count,), 1.0, seed=count)
+    xd = x.cuda()
+    s = P.act_scale(xd)
+    rs = O.tensor_scale(x.numpy())
+    assert s.item() == rs
+    q = P.quantize(xd, s)
+    assert np.array_equal(q.cpu().numpy(), O.quantize(x.numpy(), rs))
+
+
+def test_act_scale_and_quantize_int8_workload():
+    w = I.int8_long_tail()
+    xd = w.X.cuda()
+    s = P.act_scale(xd)
+    rs = O.tensor_scale(w.X.numpy())
+    assert s.item() == rs
+    q = P.quantize(xd, s)
+    rows = np.arange(0, w.M, 97)
+    assert np.array_equal(q.cpu().numpy()[rows], O.quantize(w.X.numpy()[rows], rs))
+
+
+# ------------------------------------------------------------------ a6 bf16
+def _bf16_pipeline(W, X, mode=B.SP24_MAGNITUDE, Xc=None):
+    Wd = W.cuda()
+    mask = P.prune(Wd, mode, 2, Xc=None if Xc is None else Xc.cuda())
+    vals, meta = P.compress(Wd, mask, B.SP24_BF16)
+    y = P.gemm(X.cuda(), vals, meta, W.shape[0])
+    return mask, vals, meta, y
+
+
+def _bf16_ref(W, X, rows=None, mode=O.MAGNITUDE, Xc=None):
+    keep = O.prune(f64(W), mode, 2, xc=None if Xc is None else f64(Xc))
+    vals, meta = O.compress(f64(W), keep)
+    x = f64(X) if rows is None else f64(X[rows])
+    return O.gemm(x, vals, meta, W.shape[1])
+
+
+GEMM_SHAPES = [
+    # (M, N, K): several tiles, ragged tails in every dimension, minimal sizes
+    (16, 64, 128), (77, 72, 144), (1, 8, 16), (130, 136, 272), (300, 256, 512),
+    (33, 384, 1024), (64, 128, 256), (5, 11008, 256), (129, 4096, 384),
+]
+
+
+@pytest.mark.parametrize("mnk", GEMM_SHAPES)
+def test_gemm_bf16_shapes(mnk):
+    m, n, k = mnk
+    W = I.normal_bf16((n, k), 1.0, seed=21)
+    X = I.normal_bf16((m, k), 1.0, seed=22)
+    _, _, _, y = _bf16_pipeline(W, X)
+    yr, ar = _bf16_ref(W, X)
+    assert_bf16_close(y, yr, ar)
+    ok_status()
+
+
+def test_gemm_bf16_tiny_config():
+    w = I.tiny()
+    _, _, _, y = _bf16_pipeline(w.W, w.X)
+    assert_bf16_close(y, *_bf16_ref(w.W, w.X))
+
+
+def test_gemm_bf16_bert_full():
+    w = I.bert_fc1()
+    Wd, Xc = w.W.cuda(), w.Xc.cuda()
+    m1 = P.prune(Wd, B.SP24_WANDA, 3, Xc=Xc)
+    m2 = P.prune(Wd, B.SP24_WANDA, 2, Xc=Xc, mask_in=m1)
+    vals, meta = P.compress(Wd, m2, B.SP24_BF16)
+    y = P.gemm(w.X.cuda(), vals, meta, w.N)
+    keep = O.progressive(f64(w.W), O.WANDA, f64(w.Xc))[1]
+    rv, rm = O.compress(f64(w.W), keep)
+    assert_bf16_close(y, *O.gemm(f64(w.X), rv, rm, w.K))
+
+
+@pytest.mark.parametrize("nk", I.LLM_SHAPES)
+@pytest.mark.parametrize("m", I.LLM_M)
+def test_gemm_bf16_llm(nk, m):
+    n, k = nk
+    w = I.llm_proj(n, k, m)
+    _, _, _, y = _bf16_pipeline(w.W, w.X)
+    rows = np.arange(m) if m <= 128 else np.unique(np.r_[0:8, m - 8:m, 97:m:211])
+    yr, ar = _bf16_ref(w.W, w.X, rows)
+    assert_bf16_close(y[torch.from_numpy(rows).cuda()], yr, ar)
+
+
+def test_gemm_bf16_conv1x1_sampled():
+    w = I.conv1x1()
+    _, _, _, y = _bf16_pipeline(w.W, w.X)
+    rows = np.unique(np.r_[0:64, w.M - 64:w.M, 1000:w.M:4093])
+    yr, ar = _bf16_ref(w.W, w.X, rows)
+    assert_bf16_close(y[torch.from_numpy(rows).cuda()], yr, ar)
+
+
+@pytest.mark.parametrize("n", [1024, 4096])
+def test_gemm_bf16_square(n):
+    w = I.square(n)
+    _, _, _, y = _bf16_pipeline(w.W, w.X)
+    rows = np.arange(n) if n <= 1024 else np.unique(np.r_[0:16, n - 16:n, 100:n:257])
+    yr, ar = _bf16_ref(w.W, w.X, rows)
+    assert_bf16_close(y[torch.from_numpy(rows).cuda()], yr, ar)
+
+
+def test_gemm_bf16_deterministic_split():
+    w = I.llm_proj(4096, 11008, 16)      # split-K over a cluster
+    _, vals, meta, y1 = _bf16_pipeline(w.W, w.X)
+    y2 = P.gemm(w.X.cuda(), vals, meta, w.N)
+    assert torch.equal(y1, y2)
+
+
+def test_gemm_empty_is_noop():
+    W = I.normal_bf16((64, 128), 1.0, seed=1).cuda()
+    mask = P.prune(W, B.SP24_MAGNITUDE, 2)
+    vals, meta = P.compress(W, mask)
+    y = P.gemm(torch.empty((0, 128), dtype=torch.bfloat16, device="cuda"), vals, meta, 64)
+    assert y.shape == (0, 64)
+    ok_status()
+
+
+# ------------------------------------------------------------------ a7 int8
+def _int8_pipeline(W, X32, out_kind, s_y=None):
+    Wd = W.cuda()
+    mask = P.prune(Wd, B.SP24_MAGNITUDE, 2)
+    s_w = P.wscale(Wd, mask)
+    vals, meta = P.compress(Wd, mask, B.SP24_INT8, s_w)
+    xd = X32.cuda()
+    s_x = P.act_scale(xd)
+    xq = P.quantize(xd, s_x)
+    sy = None if s_y is None else torch.tensor([s_y], dtype=torch.float32, device="cuda")
+    y = P.gemm(xq, vals, meta, W.shape[0], B.SP24_INT8, s_x, s_w, out_kind, sy)
+    return y, s_x.item(), s_w.cpu().numpy()
+
+
+def _int8_ref(W, X32, rows=None):
+    keep = O.prune(f64(W), O.MAGNITUDE, 2)
+    s_w = O.channel_scales(f64(W), keep)
+    vq, meta = O.compress(O.quantize(f64(W), s_w[:, None]), keep)
+    s_x = O.tensor_scale(X32.numpy())
+    x = X32.numpy() if rows is None else X32.numpy()[rows]
+    acc = O.gemm_int8_acc(O.quantize(x, s_x), vq, meta, W.shape[1])
+    return acc, s_x, s_w
+
+
+INT8_SHAPES = [(16, 64, 128), (77, 72, 160), (1, 8, 32), (130, 136, 288), (300, 256, 512),
+               (16, 11008, 4096), (128, 4096, 1024)]
+
+
+@pytest.mark.parametrize("mnk", INT8_SHAPES)
+def test_gemm_int8_shapes(mnk):
+    m, n, k = mnk
+    W = I.long_tail_bf16((n, k), 0.02, seed=31, tail_seed=34)
+    X = I.normal_f32((m, k), 1.0, seed=32)
+    acc, s_x, s_w = _int8_ref(W, X)
+    y32, gx, gw = _int8_pipeline(W, X, B.SP24_OUT_INT32)
+    assert gx == s_x and np.array_equal(gw, s_w)
+    assert np.array_equal(y32.cpu().numpy(), acc)
+    ybf, _, _ = _int8_pipeline(W, X, B.SP24_OUT_BF16)
+    ref_bits = O.dequant_bf16(acc, s_x, s_w)
+    assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), ref_bits)
+    y8, _, _ = _int8_pipeline(W, X, B.SP24_OUT_INT8, s_y=0.05)
+    assert np.array_equal(y8.cpu().numpy(), O.requant_int8(acc, s_x, s_w, np.float32(0.05)))
+    ok_status()
+
+
+def test_gemm_int8_full_config_sampled():
+    w = I.int8_long_tail()
+    rows = np.unique(np.r_[0:8, w.M - 8:w.M, 51:w.M:397])
+    acc, s_x, s_w = _int8_ref(w.W, w.X, rows)
+    ybf, gx, gw = _int8_pipeline(w.W, w.X, B.SP24_OUT_BF16)
+    assert gx == s_x and np.array_equal(gw, s_w)
+    got = ybf[torch.from_numpy(rows).cuda()].view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, O.dequant_bf16(acc, s_x, s_w))
+    y32, _, _ = _int8_pipeline(w.W, w.X, B.SP24_OUT_INT32)
+    assert np.array_equal(y32[torch.from_numpy(rows).cuda()].cpu().numpy(), acc)
+    ok_status()
