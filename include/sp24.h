@@ -113,7 +113,9 @@ sp24_status sp24_colnorm(const void* Xc, int64_t Mc, int64_t K, double* norms,
  * remaining weights).
  *   W: bf16 [N][K].  Xc: bf16 [Mc][K] (SP24_WANDA only, else ignored).
  *   mask_in (nullable), mask_out: sp24_mask_bytes(N, K) bytes.
- *   workspace: sp24_prune_workspace_bytes(K, mode) bytes (NULL if 0).
+ *   workspace: sp24_prune_workspace_bytes(K, mode) bytes (NULL if 0).  For
+ *              SP24_WANDA it holds the float64 column norms [K] afterwards,
+ *              ready to pass as `norms` to sp24_prune_compress.
  * Rules: N >= 0, K % 8 == 0, n_keep in {2, 3}; Mc >= 1 for SP24_WANDA. */
 sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc,
                        int64_t Mc, int mode, int n_keep, const uint8_t* mask_in,
@@ -127,7 +129,7 @@ sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc,
  * in IEEE double; s_w[n] = float(t_n) / 127.0f (float32 divide), or 1 when
  * t_n == 0.  For c <= 9999 and coverage 0.9999 this is the row maximum.
  *   W: bf16 [N][K].  mask: sp24_mask_bytes(N, K) bytes.  s_w: float32 [N].
- * Rules: K % 8 == 0, 0 < coverage <= 1, K/2 <= 65536. */
+ * Rules: K % 8 == 0, 0 < coverage <= 1. */
 sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K,
                         double coverage, float* s_w, void* stream);
 
@@ -192,7 +194,8 @@ sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
  *       -127, 127), float32 divide.
  *       s_x, s_y: one float32 each (device); s_w: float32 [N] (device).
  * vals/meta come from sp24_compress with the same dtype, N and K.
- * Rules: M >= 0, N >= 0, N % 8 == 0; K >= 16, K % 16 == 0 (bf16) or
+ * Rules: M >= 0, N >= 0, N % 8 == 0 (N % 16 == 0 for SP24_OUT_INT8, so that
+ * rows of Y stay 16-byte aligned); K >= 16, K % 16 == 0 (bf16) or
  * K % 32 == 0 (int8); alignment of 16 bytes for every pointer.  Ragged M, N
  * and K tails are handled in the kernel (no padding copies; [Orin ch.7] 6.2). */
 sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
@@ -209,6 +212,12 @@ sp24_status sp24_device_status(void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* sp24_strerror(int status);
+
+/* Text naming the last CUDA runtime / driver call that failed inside a libsp24
+ * entry point on the calling thread and its error (e.g. "kernel launch:
+ * cudaErrorInvalidValue"), or "" if none has failed.  Valid until the next
+ * libsp24 call on this thread. */
+const char* sp24_last_cuda_error(void);
 
 /* Library version: major*10000 + minor*100 + patch. */
 int sp24_version(void);

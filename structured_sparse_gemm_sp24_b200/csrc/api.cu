@@ -1,4 +1,5 @@
 // libsp24: size queries, status word, error strings, device checks.
+#include <cstdio>
 #include <mutex>
 
 #include "sp24_device.cuh"
@@ -13,16 +14,27 @@ int g_dev_sms[kMaxDevices];
 std::mutex g_dev_mu;
 }  // namespace
 
+namespace {
+thread_local char g_last_err[256] = "";
+}  // namespace
+
+sp24_status cuda_fail(const char* what, const char* err_name) {
+  std::snprintf(g_last_err, sizeof(g_last_err), "%s: %s", what, err_name ? err_name : "?");
+  return SP24_ERR_CUDA;
+}
+
 sp24_status check_device() {
+  g_last_err[0] = '\0';
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SP24_ERR_CUDA;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return SP24_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_dev_mu);
   if (g_dev_ok[dev] == 0) {
     int major = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return SP24_ERR_CUDA;
+    cudaError_t a = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (a == cudaSuccess) a = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (a != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", a);
     g_dev_ok[dev] = (major == 10) ? 1 : 2;
     g_dev_sms[dev] = sms;
   }
@@ -66,12 +78,16 @@ size_t sp24_prune_workspace_bytes(int64_t K, int mode) {
 }
 
 sp24_status sp24_device_status(void* stream) {
-  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SP24_ERR_CUDA;
+  g_last_err[0] = '\0';
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail("cudaStreamSynchronize", e);
   uint32_t word = 0;
-  if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return SP24_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&word, g_status, sizeof(word));
+  if (e != cudaSuccess) return cuda_fail("cudaMemcpyFromSymbol", e);
   if (word != 0) {
     const uint32_t zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SP24_ERR_CUDA;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail("cudaMemcpyToSymbol", e);
   }
   if (word & kErrTimeoutBit) return SP24_ERR_TIMEOUT;
   if (word & kErrPatternBit) return SP24_ERR_PATTERN;
@@ -92,5 +108,7 @@ const char* sp24_strerror(int status) {
 }
 
 int sp24_version(void) { return 100; }
+
+const char* sp24_last_cuda_error(void) { return g_last_err; }
 
 }  // extern "C"

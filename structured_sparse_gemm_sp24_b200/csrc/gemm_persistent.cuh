@@ -1,0 +1,281 @@
+// Persistent, warp-specialised sparse GEMM for problems with at least one
+// output tile per SM (the tensor-core-bound regime).  Included by gemm_sp.cu.
+//
+// Same operands, metadata path and MMA issue as the split-K kernel, plus:
+//  * one CTA per SM walks a static list of 128 x BN output tiles in a grouped
+//    order: GROUP_ROWS weight row tiles are swept across all token tiles
+//    before the next group, so one group's compressed weights and the token
+//    tiles of a wave stay in L2 (each weight byte is fetched from HBM once);
+//  * two tensor-memory accumulators: the MMA warp fills one tile while the
+//    epilogue warps drain the other;
+//  * the epilogue drains 32 columns (tokens) at a time: tcgen05.ld -> cast /
+//    dequantise in registers -> shared-memory staging [32 tokens][128
+//    channels] -> TMA tensor store (clipped at the M / N edges), with two
+//    staging buffers so the store of one chunk overlaps the next.
+// Warps: 0 = TMA producer, 1 = MMA issuer, 2..5 = epilogue (warp 2 also owns
+// the tensor-memory allocation).
+#pragma once
+
+namespace sp24 {
+
+template <int kDtype, int BN, int STAGES, int OUTK>
+struct PersistCfg {
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBHalfBytes = BN * 128;
+  static constexpr int kMetaChunks = kDtype == SP24_BF16 ? 1 : 2;
+  static constexpr int kEBytes = 2048 * kMetaChunks;
+  static constexpr int kStageBytes = kABytes + 2 * kBHalfBytes + kEBytes;
+  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kLogicalK = kDtype == SP24_BF16 ? 128 : 256;
+  static constexpr int kMmaK = kLogicalK / 4;
+  static constexpr int kMetaCols = 4 * kMetaChunks;
+  static constexpr int kAcc = 2;
+  static constexpr int kMetaCol0 = kAcc * BN;
+  static constexpr int kTmemNeeded = kAcc * BN + 2 * kMetaCols;
+  static constexpr int kTmemCols = kTmemNeeded <= 32 ? 32
+                                   : kTmemNeeded <= 64 ? 64
+                                   : kTmemNeeded <= 128 ? 128
+                                   : kTmemNeeded <= 256 ? 256 : 512;
+  static constexpr int kOutBytes = OUTK == SP24_OUT_INT32 ? 4 : (OUTK == SP24_OUT_INT8 ? 1 : 2);
+  static constexpr int kChunk = 32;                              // tokens per epilogue chunk
+  // store box: [32 tokens][y_box channels], y_box = min(kChBox, N) (the
+  // tensor-map encoder rejects a box wider than the tensor), at most 256
+  // bytes per row; a staging buffer holds the boxes of one chunk back to back
+  static constexpr int kChBox = kOutBytes == 4 ? 64 : 128;
+  static constexpr int kStagingBytes = kChunk * 128 * kOutBytes;  // one staging buffer
+  static constexpr int kRingBytes = STAGES * kStageStride;
+  static constexpr int kSmemBytes = kRingBytes + 2 * kStagingBytes + 1024 + 256;
+  static_assert(kTmemNeeded <= 512, "tensor memory overflow");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+struct PersistArgs {
+  const uint8_t* meta;
+  const float* s_x;
+  const float* s_w;
+  const float* s_y;
+  int64_t m, n, k;
+  int kblocks;       // K stages per tile
+  int row_tiles;     // ceil(N / 128)
+  int tok_tiles;     // ceil(M / BN)
+  int group_rows;    // raster group height (row tiles)
+  int y_box;         // channels per TMA store box: min(kChBox, N), a multiple of 8
+};
+
+// Linear tile index -> (row tile, token tile) in the grouped order.
+__device__ __forceinline__ void tile_coords(int t, const PersistArgs& a, int& rt, int& tt) {
+  const int per_group = a.group_rows * a.tok_tiles;
+  const int g = t / per_group;
+  const int r = t - g * per_group;
+  int rows = a.row_tiles - g * a.group_rows;
+  rows = rows < a.group_rows ? rows : a.group_rows;
+  rt = g * a.group_rows + r % rows;
+  tt = r / rows;
+}
+
+template <int kDtype, int BN, int STAGES, int OUTK>
+__global__ void __launch_bounds__(192, 1)
+gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_b,
+                   const __grid_constant__ CUtensorMap tmap_y, const PersistArgs args) {
+  using C = PersistCfg<kDtype, BN, STAGES, OUTK>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* staging = smem + C::kRingBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + 2 * C::kStagingBytes);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + C::kAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + C::kAcc);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ntiles = args.row_tiles * args.tok_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < C::kAcc; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kchunks = static_cast<int>((args.k + 127) / 128);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      prefetch_tmap(&tmap_a);
+      prefetch_tmap(&tmap_b);
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        int rt, tt;
+        tile_coords(tile, args, rt, tt);
+        const uint8_t* meta_tile = args.meta + static_cast<int64_t>(rt) * kchunks * 2048;
+        for (int kb = 0; kb < args.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u)) { *abort_flag = 1; break; }
+          uint8_t* st = smem + s * C::kStageStride;
+          int chunks = C::kMetaChunks;
+          if (kDtype == SP24_INT8 && 2 * kb + 1 >= kchunks) chunks = 1;
+          mbar_arrive_expect_tx(&full_bar[s], C::kABytes + 2 * C::kBHalfBytes + 2048 * chunks);
+          tma_load_2d(st, &tmap_a, &full_bar[s], kb * (kDtype == SP24_BF16 ? 64 : 128), rt * 128);
+          const int kx = kb * C::kLogicalK;
+          tma_load_2d(st + C::kABytes, &tmap_b, &full_bar[s], kx, tt * BN);
+          tma_load_2d(st + C::kABytes + C::kBHalfBytes, &tmap_b, &full_bar[s],
+                      kx + C::kLogicalK / 2, tt * BN);
+          bulk_load(st + C::kABytes + 2 * C::kBHalfBytes,
+                    meta_tile + static_cast<int64_t>(kb * C::kMetaChunks) * 2048,
+                    2048u * chunks, &full_bar[s]);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------ MMA issuer
+      uint32_t it = 0, j = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++j) {
+        const uint32_t acc = j % C::kAcc;
+        if (!mbar_wait(&tempty_bar[acc], ((j / C::kAcc) & 1u) ^ 1u)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool aborted = false;
+        for (int kb = 0; kb < args.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full_bar[s], ph)) { *abort_flag = 1; aborted = true; break; }
+          tc_fence_after();
+          uint8_t* st = smem + s * C::kStageStride;
+          const uint32_t a_addr = smem_u32(st);
+          const uint32_t b_addr = smem_u32(st + C::kABytes);
+          const uint32_t e_addr = smem_u32(st + C::kABytes + 2 * C::kBHalfBytes);
+          const uint32_t meta_col = C::kMetaCol0 + (it & 1u) * C::kMetaCols;
+          const int64_t k_left = args.k - static_cast<int64_t>(kb) * C::kLogicalK;
+          int n_mma = static_cast<int>((k_left + C::kMmaK - 1) / C::kMmaK);
+          n_mma = n_mma > 4 ? 4 : n_mma;
+          const int chunks = kDtype == SP24_BF16 ? 1 : (n_mma > 2 ? 2 : 1);
+          for (int c = 0; c < chunks; ++c)
+            tc_cp_128x128b(tmem_base + meta_col + 4 * c,
+                           smem_desc(e_addr + 2048 * c, 128, 128, kSwizzleNone));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q < n_mma) {
+              const uint64_t a_desc = smem_desc(a_addr + 32 * q, 0, 1024, kSwizzle128B);
+              const uint64_t b_desc = smem_desc(
+                  b_addr + (q >> 1) * C::kBHalfBytes + 64 * (q & 1), 0, 1024, kSwizzle128B);
+              const uint32_t accumulate = (kb > 0 || q > 0) ? 1u : 0u;
+              if constexpr (kDtype == SP24_BF16) {
+                tc_mma_sp(d_tmem, a_desc, b_desc, tmem_base + meta_col + (q & ~1),
+                          make_idesc<kDtype, BN>(q & 1), accumulate);
+              } else {
+                tc_mma_sp_i8(d_tmem, a_desc, b_desc, tmem_base + meta_col + 2 * q,
+                             make_idesc<kDtype, BN>(0), accumulate);
+              }
+            }
+          }
+          tc_commit(&empty_bar[s]);
+        }
+        tc_commit(&tfull_bar[acc]);   // accumulator of this tile complete (or abandoned)
+        if (aborted) break;
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quad = warp & 3;               // tensor-memory lane quadrant of this warp
+    const int row = quad * 32 + lane;        // output channel within the tile
+    const int tid_e = threadIdx.x - 64;      // 0..127
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sx = (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32) ? *args.s_x : 1.0f;
+    const float sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
+    // staging element of (token 0, this channel): box row / ybox, column row % ybox
+    const int ybox = args.y_box;
+    const int sidx = (row / ybox) * (C::kChunk * ybox) + (row % ybox);
+    uint32_t j = 0, chunk_ctr = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
+      int rt, tt;
+      tile_coords(tile, args, rt, tt);
+      const uint32_t acc = j % C::kAcc;
+      bool ok = true;
+      if (tid_e == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
+      if (!named_barrier_and(1, 128, ok)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int64_t n_idx = static_cast<int64_t>(rt) * 128 + row;
+      const bool row_valid = n_idx < args.n;
+      float cscale = 0.0f;
+      if constexpr (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32)
+        cscale = n_idx < args.n ? __fmul_rn(sx, __ldg(args.s_w + n_idx)) : 0.0f;
+      const int64_t tok0 = static_cast<int64_t>(tt) * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / C::kChunk; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + acc * BN + c * C::kChunk, r);
+        tmem_ld_wait();
+        if (c == BN / C::kChunk - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[acc]);   // accumulator drained
+        }
+        if (tok0 + c * C::kChunk >= args.m) continue;       // chunk entirely past M
+        uint8_t* stg = staging + (chunk_ctr & 1u) * C::kStagingBytes;
+        if (tid_e == 0) bulk_wait_read<1>();                 // buffer's previous store done
+        named_barrier(1, 128);
+        // channels at or past N are never stored (and, when N < 128, would
+        // index past the staging buffer): skip them
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (!row_valid) break;
+          const int e = sidx + t * ybox;
+          if constexpr (kDtype == SP24_BF16) {
+            const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[t]));
+            reinterpret_cast<__nv_bfloat16*>(stg)[e] = h;
+          } else if constexpr (OUTK == SP24_OUT_INT32) {
+            reinterpret_cast<uint32_t*>(stg)[e] = r[t];
+          } else {
+            const float f = __fmul_rn(__int2float_rn(static_cast<int32_t>(r[t])), cscale);
+            if constexpr (OUTK == SP24_OUT_BF16) {
+              reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(f);
+            } else {
+              int qv = __float2int_rn(__fdiv_rn(f, sy));
+              qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
+              reinterpret_cast<int8_t*>(stg)[e] = static_cast<int8_t>(qv);
+            }
+          }
+        }
+        fence_async_shared();
+        named_barrier(1, 128);
+        if (tid_e == 0) {
+          for (int bx = 0; bx * ybox < 128 && rt * 128 + bx * ybox < args.n; ++bx)
+            tma_store_2d(&tmap_y, stg + bx * (C::kChunk * ybox * C::kOutBytes),
+                         rt * 128 + bx * ybox, static_cast<int32_t>(tok0 + c * C::kChunk));
+          bulk_commit();
+        }
+        ++chunk_ctr;
+      }
+    }
+    if (tid_e == 0) bulk_wait<0>();
+  }
+
+  __syncwarp();
+  if (*abort_flag) settle_ns(20000);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+}  // namespace sp24

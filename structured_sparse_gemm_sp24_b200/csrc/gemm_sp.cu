@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "sp24_device.cuh"
@@ -310,6 +311,12 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
   if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+}  // namespace sp24
+
+#include "gemm_persistent.cuh"
+
+namespace sp24 {
+
 // ----------------------------------------------------------------- host side
 namespace {
 
@@ -330,16 +337,23 @@ bool get_encoder() {
 
 // 2D row-major [rows][cols] map with a {box_cols, box_rows} box, 128B swizzle,
 // zero fill outside the tensor.
-bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elsize,
-              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+sp24_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elsize,
+              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elsize)};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  return g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                             CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r == CUDA_SUCCESS) return SP24_OK;
+  char buf[96];
+  std::snprintf(buf, sizeof(buf), "CUresult %d (box %ux%u, dims %llux%llu)", static_cast<int>(r),
+                box_cols, box_rows, static_cast<unsigned long long>(cols),
+                static_cast<unsigned long long>(rows));
+  return cuda_fail("cuTensorMapEncodeTiled", buf);
 }
 
 template <int kDtype, int BN, int STAGES, int SPLIT>
@@ -349,12 +363,12 @@ sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const 
   auto kern = gemm_sp_kernel<kDtype, BN, STAGES, SPLIT>;
   static uint64_t attr_set = 0;   // one bit per device (devices 0..63)
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SP24_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return SP24_ERR_CUDA;
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
     attr_set |= bit;
   }
   const int64_t row_tiles = (a.n + 127) / 128;
@@ -372,7 +386,56 @@ sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, ma, mb, a) != cudaSuccess) return SP24_ERR_CUDA;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, a);
+  if (le != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", le);
+  return launch_status();
+}
+
+
+template <int kDtype, int BN, int STAGES, int OUTK>
+sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                              cudaStream_t s) {
+  using C = PersistCfg<kDtype, BN, STAGES, OUTK>;
+  auto kern = gemm_sp_persistent<kDtype, BN, STAGES, OUTK>;
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    attr_set |= bit;
+  }
+  const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                  : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int y_box = static_cast<int>(g.n < C::kChBox ? g.n : C::kChBox);
+  CUtensorMap my;
+  SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), C::kChunk,
+                    CU_TENSOR_MAP_SWIZZLE_NONE));
+  PersistArgs a;
+  a.meta = g.meta;
+  a.s_x = g.s_x;
+  a.s_w = g.s_w;
+  a.s_y = g.s_y;
+  a.m = g.m;
+  a.n = g.n;
+  a.k = g.k;
+  a.kblocks = g.kblocks;
+  a.row_tiles = static_cast<int>((g.n + 127) / 128);
+  a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
+  // raster group: as many weight row tiles as fit ~24 MB of compressed weights
+  const int64_t row_tile_bytes = 128 * (g.k / 2) * (kDtype == SP24_BF16 ? 2 : 1);
+  int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
+  a.group_rows = static_cast<int>(gr);
+  a.y_box = y_box;
+  const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
+  if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(ntiles < sm_count() ? ntiles : sm_count());
+  kern<<<grid, 192, C::kSmemBytes, s>>>(ma, mb, my, a);
   return launch_status();
 }
 
@@ -393,12 +456,20 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
       kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint32_t box_cols = 128 / el;
   CUtensorMap ma, mb;
-  if (!make_map(&ma, vals, dt, el, static_cast<uint64_t>(a.k / 2), static_cast<uint64_t>(a.n),
-                box_cols, 128))
-    return SP24_ERR_CUDA;
-  if (!make_map(&mb, x, dt, el, static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.m), box_cols,
-                static_cast<uint32_t>(bn)))
-    return SP24_ERR_CUDA;
+  SP24_TRY(make_map(&ma, vals, dt, el, static_cast<uint64_t>(a.k / 2),
+                    static_cast<uint64_t>(a.n), box_cols, 128));
+  SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.m),
+                    box_cols, static_cast<uint32_t>(bn)));
+
+  if (split == 1 && bn == 128) {
+    if constexpr (kDtype == SP24_BF16) {
+      return launch_persistent<kDtype, 128, 4, SP24_OUT_BF16>(ma, mb, a, s);
+    } else {
+      if (a.out_kind == SP24_OUT_INT32) return launch_persistent<kDtype, 128, 3, SP24_OUT_INT32>(ma, mb, a, s);
+      if (a.out_kind == SP24_OUT_INT8) return launch_persistent<kDtype, 128, 4, SP24_OUT_INT8>(ma, mb, a, s);
+      return launch_persistent<kDtype, 128, 4, SP24_OUT_BF16>(ma, mb, a, s);
+    }
+  }
 
 #define SP24_GEMM_CASE(BN_, ST_)                                                          \
   if (bn == BN_) {                                                                        \
@@ -436,13 +507,14 @@ extern "C" sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void
   if (dtype == SP24_INT8 && out_kind != SP24_OUT_INT32 && (!s_x || !s_w)) return SP24_ERR_ARG;
   if (dtype == SP24_INT8 && out_kind == SP24_OUT_INT8 && !s_y) return SP24_ERR_ARG;
   if (K < 16 || N % 8 != 0 || K % (dtype == SP24_BF16 ? 16 : 32) != 0) return SP24_ERR_ALIGN;
+  if (out_kind == SP24_OUT_INT8 && dtype == SP24_INT8 && N % 16 != 0) return SP24_ERR_ALIGN;
   if (!aligned16(X) || !aligned16(vals) || !aligned16(meta) || !aligned16(Y) ||
       (s_w && !aligned16(s_w)))
     return SP24_ERR_ALIGN;
   if (K > (int64_t(1) << 31) || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
     return SP24_ERR_UNSUPPORTED;
   SP24_TRY(check_device());
-  if (!get_encoder()) return SP24_ERR_CUDA;
+  if (!get_encoder()) return cuda_fail("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled");
   GemmArgs a;
   a.meta = static_cast<const uint8_t*>(meta);
   a.s_x = s_x;

@@ -74,29 +74,35 @@ __device__ __forceinline__ uint32_t mask_byte(const uint4& w, uint32_t in, const
 }
 
 // -------------------------------------------------------------- a1 colnorm
-// Thread per 8 columns; sequential float64 sum over the Mc rows.
+// Block per 64 columns.  Each pass stages a [128 tokens][64 columns] bf16 tile
+// in shared memory with every 16-byte load in flight, then threads 0..63 add
+// the squares of their column sequentially in token order (float64, one
+// rounding per addition; the square of a bf16 value is exact).
 __global__ void __launch_bounds__(256) colnorm_kernel(const uint16_t* __restrict__ xc,
                                                       int64_t mc, int64_t k,
                                                       double* __restrict__ norms) {
-  const int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nv = k / 8;
-  if (v >= nv) return;
-  double acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0;
-  const uint4* p = reinterpret_cast<const uint4*>(xc) + v;
-  for (int64_t t = 0; t < mc; ++t) {
-    const uint4 q = __ldg(p + t * nv);
-    const uint32_t words[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t bits = (i & 1) ? (words[i / 2] >> 16) : (words[i / 2] & 0xFFFFu);
-      const double x = bf16_to_double(bits);
-      acc[i] = __dadd_rn(acc[i], __dmul_rn(x, x));  // square exact, one rounding per add
+  __shared__ __align__(16) uint16_t tile[128][64];
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 64;
+  const int cvalid = static_cast<int>(k - col0 < 64 ? k - col0 : 64);   // multiple of 8
+  double acc = 0.0;
+  for (int64_t t0 = 0; t0 < mc; t0 += 128) {
+    const int rows = static_cast<int>(mc - t0 < 128 ? mc - t0 : 128);
+    for (int i = threadIdx.x; i < rows * 8; i += blockDim.x) {
+      const int r = i >> 3, c8 = (i & 7) * 8;
+      if (c8 < cvalid)
+        *reinterpret_cast<uint4*>(&tile[r][c8]) =
+            __ldg(reinterpret_cast<const uint4*>(xc + (t0 + r) * k + col0 + c8));
     }
+    __syncthreads();
+    if (threadIdx.x < cvalid) {
+      for (int r = 0; r < rows; ++r) {
+        const double x = bf16_to_double(tile[r][threadIdx.x]);
+        acc = __dadd_rn(acc, __dmul_rn(x, x));
+      }
+    }
+    __syncthreads();
   }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) norms[8 * v + i] = __dsqrt_rn(acc[i]);
+  if (threadIdx.x < cvalid) norms[col0 + threadIdx.x] = __dsqrt_rn(acc);
 }
 
 // ------------------------------------------------------------ a2+a3 prune
@@ -439,8 +445,7 @@ static int grid_for(int64_t work_items, int threads) {
 
 static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double* norms,
                                   cudaStream_t s) {
-  const int64_t nv = k / 8;
-  const int blocks = static_cast<int>((nv + 255) / 256);
+  const int blocks = static_cast<int>((k + 63) / 64);
   colnorm_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(xc), mc, k, norms);
   return launch_status();
 }

@@ -18,9 +18,17 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 // SP24_OK when the current device is an sm_100 part (cached per device).
 sp24_status check_device();
 
+// Records a failed CUDA call for sp24_last_cuda_error() (thread-local) and
+// returns SP24_ERR_CUDA.
+sp24_status cuda_fail(const char* what, const char* err_name);
+inline sp24_status cuda_fail(const char* what, cudaError_t e) {
+  return cuda_fail(what, cudaGetErrorName(e));
+}
+
 // Maps the launch status of the last kernel to a library status.
 inline sp24_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? SP24_OK : SP24_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SP24_OK : cuda_fail("kernel launch", e);
 }
 
 // Number of SMs of the current device (cached).

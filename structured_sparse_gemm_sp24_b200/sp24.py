@@ -60,6 +60,7 @@ SIGNATURES = {
     "sp24_device_status": (_c_int, [_c_p]),
     "sp24_strerror": (ctypes.c_char_p, [_c_int]),
     "sp24_version": (_c_int, []),
+    "sp24_last_cuda_error": (ctypes.c_char_p, []),
 }
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -68,7 +69,10 @@ _LIB: Optional[ctypes.CDLL] = None
 class Sp24Error(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = int(status)
-        super().__init__(f"{where}: {strerror(status)} (status {status})")
+        detail = ""
+        if self.status == SP24_ERR_CUDA:
+            detail = " [" + lib().sp24_last_cuda_error().decode() + "]"
+        super().__init__(f"{where}: {strerror(status)} (status {status}){detail}")
 
 
 def lib() -> ctypes.CDLL:

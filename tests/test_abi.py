@@ -115,6 +115,9 @@ def test_compress_and_gemm_host_validation(lib):
              FAKE, None) == B.SP24_ERR_ARG
     assert g(FAKE, 16, 128, FAKE, FAKE, 16, B.SP24_INT8, FAKE, FAKE, B.SP24_OUT_INT8, None,
              FAKE, None) == B.SP24_ERR_ARG
+    # int8 output needs N % 16 == 0 (16-byte aligned rows)
+    assert g(FAKE, 16, 128, FAKE, FAKE, 24, B.SP24_INT8, FAKE, FAKE, B.SP24_OUT_INT8, FAKE,
+             FAKE, None) == B.SP24_ERR_ALIGN
     # empty problems
     assert g(None, 0, 128, None, None, 16, B.SP24_BF16, None, None, B.SP24_OUT_BF16, None,
              None, None) == B.SP24_OK

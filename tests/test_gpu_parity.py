@@ -267,6 +267,10 @@ GEMM_SHAPES = [
     # (M, N, K): several tiles, ragged tails in every dimension, minimal sizes
     (16, 64, 128), (77, 72, 144), (1, 8, 16), (130, 136, 272), (300, 256, 512),
     (33, 384, 1024), (64, 128, 256), (5, 11008, 256), (129, 4096, 384),
+    # persistent path (>= 2 tiles per SM, or a single K block), ragged M, N, K
+    (2500, 2056, 400), (300, 256, 128), (4099, 1032, 784),
+    # persistent path with N < 128 (store box narrower than a tile)
+    (300, 24, 128), (1000, 40, 96),
 ]
 
 
@@ -368,7 +372,9 @@ def _int8_ref(W, X32, rows=None):
 
 
 INT8_SHAPES = [(16, 64, 128), (77, 72, 160), (1, 8, 32), (130, 136, 288), (300, 256, 512),
-               (16, 11008, 4096), (128, 4096, 1024)]
+               (16, 11008, 4096), (128, 4096, 1024),
+               # persistent path, ragged M, N, K
+               (2500, 2056, 416), (300, 256, 224), (300, 40, 224), (300, 48, 224)]
 
 
 @pytest.mark.parametrize("mnk", INT8_SHAPES)
@@ -383,8 +389,14 @@ def test_gemm_int8_shapes(mnk):
     ybf, _, _ = _int8_pipeline(W, X, B.SP24_OUT_BF16)
     ref_bits = O.dequant_bf16(acc, s_x, s_w)
     assert np.array_equal(ybf.view(torch.int16).cpu().numpy().view(np.uint16), ref_bits)
-    y8, _, _ = _int8_pipeline(W, X, B.SP24_OUT_INT8, s_y=0.05)
-    assert np.array_equal(y8.cpu().numpy(), O.requant_int8(acc, s_x, s_w, np.float32(0.05)))
+    if n % 16:
+        # int8 rows of N bytes must stay 16-byte aligned
+        with pytest.raises(B.Sp24Error) as e:
+            _int8_pipeline(W, X, B.SP24_OUT_INT8, s_y=0.05)
+        assert e.value.status == B.SP24_ERR_ALIGN
+    else:
+        y8, _, _ = _int8_pipeline(W, X, B.SP24_OUT_INT8, s_y=0.05)
+        assert np.array_equal(y8.cpu().numpy(), O.requant_int8(acc, s_x, s_w, np.float32(0.05)))
     ok_status()
 
 
