@@ -1,0 +1,269 @@
+// Persistent sparse GEMM on CTA pairs (tcgen05 cta_group::2).  Included by
+// gemm_sp.cu.
+//
+// A cluster of two CTAs on two SMs computes 256 (output channels) x BN
+// (tokens) tiles.  Each CTA stages its own 128 weight rows (A), its own BN/2
+// token rows (B) and its rows' metadata; the even CTA issues one M = 256
+// tcgen05.mma.sp per 32 (bf16) / 64 (int8) K-positions that reads both CTAs'
+// shared memory and accumulates into both CTAs' tensor memory.  Against a
+// 128 x 128 tile on one SM this halves the shared-memory traffic (TMA writes
+// plus tensor-core reads) per multiply-add, which is what bounds the
+// single-SM version.
+//
+// Synchronisation:
+//  * both CTAs' TMA loads complete on the even CTA's full barrier (its
+//    producer arms it with the bytes of both CTAs);
+//  * the even CTA's MMA commits arrive on the empty barrier of both CTAs
+//    (multicast), so each producer refills its own stage;
+//  * tensor-memory full: multicast commit to both epilogues; tensor-memory
+//    empty: the even CTA's barrier collects one arrival per epilogue warp of
+//    both CTAs.
+// Warps: 0 = TMA producer (both CTAs), 1 = MMA issuer (even CTA), 2..5 =
+// epilogue (both CTAs; warp 2 also owns the tensor-memory allocation).
+#pragma once
+
+namespace sp24 {
+
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
+struct PairCfg {
+  static constexpr int kHalfN = BN / 2;                          // token rows per CTA
+  static constexpr int kABytes = 128 * 128;
+  static constexpr int kBHalfBytes = kHalfN * 128;               // one K-half of B
+  static constexpr int kMetaChunks = kDtype == SP24_BF16 ? 1 : 2;
+  static constexpr int kEBytes = 2048 * kMetaChunks;
+  static constexpr int kStageBytes = kABytes + 2 * kBHalfBytes + kEBytes;
+  static constexpr int kStageStride = (kStageBytes + 1023) / 1024 * 1024;
+  static constexpr int kLogicalK = kDtype == SP24_BF16 ? 128 : 256;
+  static constexpr int kMmaK = kLogicalK / 4;
+  static constexpr int kMetaCols = 4 * kMetaChunks;
+  static constexpr int kAcc = ACC;
+  static constexpr int kMetaCol0 = kAcc * BN;
+  static constexpr int kTmemNeeded = kAcc * BN + 2 * kMetaCols;
+  static constexpr int kTmemCols = kTmemNeeded <= 32 ? 32
+                                   : kTmemNeeded <= 64 ? 64
+                                   : kTmemNeeded <= 128 ? 128
+                                   : kTmemNeeded <= 256 ? 256 : 512;
+  static constexpr int kOutBytes = OUTK == SP24_OUT_INT32 ? 4 : (OUTK == SP24_OUT_INT8 ? 1 : 2);
+  static constexpr int kChunk = 32;
+  static constexpr int kChBox = kOutBytes == 4 ? 64 : 128;
+  static constexpr int kStagingBytes = kChunk * 128 * kOutBytes;
+  static constexpr int kRingBytes = STAGES * kStageStride;
+  static constexpr int kSmemBytes = kRingBytes + 2 * kStagingBytes + 1024 + 256;
+  static_assert(kTmemNeeded <= 512, "tensor memory overflow");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+// Instruction descriptor for M = 256 (pair) sparse MMAs.
+template <int kDtype, int BN>
+__device__ __forceinline__ uint32_t make_idesc_pair(uint32_t id2) {
+  const uint32_t c_fmt = kDtype == SP24_BF16 ? 1u : 2u;
+  return (id2 & 3u) | (1u << 2) | (c_fmt << 4) | (1u << 7) | (1u << 10) |
+         (static_cast<uint32_t>(BN >> 3) << 17) | ((256u >> 4) << 24);
+}
+
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
+__global__ void __launch_bounds__(192, 1)
+gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+             const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
+             const PersistArgs args) {
+  using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* staging = smem + C::kRingBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + 2 * C::kStagingBytes);
+  uint64_t* empty_bar = full_bar + STAGES;
+  uint64_t* tfull_bar = empty_bar + STAGES;
+  uint64_t* tempty_bar = tfull_bar + C::kAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + C::kAcc);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();            // 0 = even (MMA-issuing) CTA
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+  const int ntiles = args.row_tiles * args.tok_tiles;  // row tiles of 256 here
+  const int kchunks = static_cast<int>((args.k + 127) / 128);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < C::kAcc; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 8);   // 4 epilogue warps x 2 CTAs
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();          // barriers of both CTAs initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------- producer
+      prefetch_tmap(&tmap_a);
+      prefetch_tmap(&tmap_b);
+      prefetch_tmap(&tmap_e);
+      uint32_t it = 0;
+      for (int tile = pair; tile < ntiles && !*abort_flag; tile += npairs) {
+        int prt, tt;
+        tile_coords(tile, args, prt, tt);
+        const int rt128 = prt * 2 + static_cast<int>(rank);   // this CTA's 128-row tile
+        for (int kb = 0; kb < args.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u)) { *abort_flag = 1; break; }
+          uint8_t* st = smem + s * C::kStageStride;
+          const uint32_t fb = map_peer(smem_u32(&full_bar[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full_bar[s], 2u * C::kStageBytes);
+          tma_load_2d_pair(st, &tmap_a, fb, kb * (kDtype == SP24_BF16 ? 64 : 128), rt128 * 128);
+          const int kx = kb * C::kLogicalK;
+          const int ty = tt * BN + static_cast<int>(rank) * C::kHalfN;
+          tma_load_2d_pair(st + C::kABytes, &tmap_b, fb, kx, ty);
+          tma_load_2d_pair(st + C::kABytes + C::kBHalfBytes, &tmap_b, fb, kx + C::kLogicalK / 2,
+                           ty);
+          // metadata map: 8 rows of 256 bytes per 2048-byte chunk
+          tma_load_2d_pair(st + C::kABytes + 2 * C::kBHalfBytes, &tmap_e, fb, 0,
+                           (rt128 * kchunks + kb * C::kMetaChunks) * 8);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ------------------------------------------------------ MMA issuer
+      uint32_t it = 0, j = 0;
+      for (int tile = pair; tile < ntiles && !*abort_flag; tile += npairs, ++j) {
+        const uint32_t acc = j % C::kAcc;
+        if (!mbar_wait(&tempty_bar[acc], ((j / C::kAcc) & 1u) ^ 1u)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        bool aborted = false;
+        for (int kb = 0; kb < args.kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full_bar[s], ph)) { *abort_flag = 1; aborted = true; break; }
+          tc_fence_after();
+          uint8_t* st = smem + s * C::kStageStride;
+          const uint32_t a_addr = smem_u32(st);
+          const uint32_t b_addr = smem_u32(st + C::kABytes);
+          const uint32_t e_addr = smem_u32(st + C::kABytes + 2 * C::kBHalfBytes);
+          const uint32_t meta_col = C::kMetaCol0 + (it & 1u) * C::kMetaCols;
+          const int64_t k_left = args.k - static_cast<int64_t>(kb) * C::kLogicalK;
+          int n_mma = static_cast<int>((k_left + C::kMmaK - 1) / C::kMmaK);
+          n_mma = n_mma > 4 ? 4 : n_mma;
+          for (int c = 0; c < C::kMetaChunks; ++c)
+            tc_cp_128x128b_pair(tmem_base + meta_col + 4 * c,
+                                smem_desc(e_addr + 2048 * c, 128, 128, kSwizzleNone));
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q < n_mma) {
+              const uint64_t a_desc = smem_desc(a_addr + 32 * q, 0, 1024, kSwizzle128B);
+              const uint64_t b_desc = smem_desc(
+                  b_addr + (q >> 1) * C::kBHalfBytes + 64 * (q & 1), 0, 1024, kSwizzle128B);
+              const uint32_t accumulate = (kb > 0 || q > 0) ? 1u : 0u;
+              if constexpr (kDtype == SP24_BF16) {
+                tc_mma_sp_pair(d_tmem, a_desc, b_desc, tmem_base + meta_col + (q & ~1),
+                               make_idesc_pair<kDtype, BN>(q & 1), accumulate);
+              } else {
+                tc_mma_sp_i8_pair(d_tmem, a_desc, b_desc, tmem_base + meta_col + 2 * q,
+                                  make_idesc_pair<kDtype, BN>(0), accumulate);
+              }
+            }
+          }
+          tc_commit_pair_mc(&empty_bar[s], 0x3);   // frees the stage in both CTAs
+        }
+        tc_commit_pair_mc(&tfull_bar[acc], 0x3);   // both epilogues may drain
+        if (aborted) break;
+      }
+    }
+  } else {
+    // --------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int tid_e = threadIdx.x - 64;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const float sx = (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32) ? *args.s_x : 1.0f;
+    const float sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
+    const int ybox = args.y_box;
+    const int sidx = (row / ybox) * (C::kChunk * ybox) + (row % ybox);
+    uint32_t j = 0, chunk_ctr = 0;
+    for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
+      int prt, tt;
+      tile_coords(tile, args, prt, tt);
+      const int rt128 = prt * 2 + static_cast<int>(rank);
+      const uint32_t acc = j % C::kAcc;
+      bool ok = true;
+      if (tid_e == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
+      if (!named_barrier_and(1, 128, ok)) { *abort_flag = 1; break; }
+      tc_fence_after();
+      const int64_t n_idx = static_cast<int64_t>(rt128) * 128 + row;
+      const bool row_valid = n_idx < args.n;
+      float cscale = 0.0f;
+      if constexpr (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32)
+        cscale = row_valid ? __fmul_rn(sx, __ldg(args.s_w + n_idx)) : 0.0f;
+      const int64_t tok0 = static_cast<int64_t>(tt) * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / C::kChunk; ++c) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + acc * BN + c * C::kChunk, r);
+        tmem_ld_wait();
+        if (c == BN / C::kChunk - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(map_peer(smem_u32(&tempty_bar[acc]), 0));
+        }
+        if (tok0 + c * C::kChunk >= args.m) continue;
+        uint8_t* stg = staging + (chunk_ctr & 1u) * C::kStagingBytes;
+        if (tid_e == 0) bulk_wait_read<1>();
+        named_barrier(1, 128);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (!row_valid) break;
+          const int e = sidx + t * ybox;
+          if constexpr (kDtype == SP24_BF16) {
+            reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(__uint_as_float(r[t]));
+          } else if constexpr (OUTK == SP24_OUT_INT32) {
+            reinterpret_cast<uint32_t*>(stg)[e] = r[t];
+          } else {
+            const float f = __fmul_rn(__int2float_rn(static_cast<int32_t>(r[t])), cscale);
+            if constexpr (OUTK == SP24_OUT_BF16) {
+              reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(f);
+            } else {
+              int qv = __float2int_rn(__fdiv_rn(f, sy));
+              qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
+              reinterpret_cast<int8_t*>(stg)[e] = static_cast<int8_t>(qv);
+            }
+          }
+        }
+        fence_async_shared();
+        named_barrier(1, 128);
+        if (tid_e == 0) {
+          for (int bx = 0; bx * ybox < 128 && rt128 * 128 + bx * ybox < args.n; ++bx)
+            tma_store_2d(&tmap_y, stg + bx * (C::kChunk * ybox * C::kOutBytes),
+                         rt128 * 128 + bx * ybox, static_cast<int32_t>(tok0 + c * C::kChunk));
+          bulk_commit();
+        }
+        ++chunk_ctr;
+      }
+    }
+    if (tid_e == 0) bulk_wait<0>();
+  }
+
+  __syncwarp();
+  if (*abort_flag) settle_ns(20000);
+  tc_fence_before();
+  cluster_sync();          // no CTA leaves while its peer may still signal it
+  if (warp == 2) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+}
+
+}  // namespace sp24

@@ -31,6 +31,8 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "sp24_device.cuh"
@@ -314,6 +316,7 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
 }  // namespace sp24
 
 #include "gemm_persistent.cuh"
+#include "gemm_pair.cuh"
 
 namespace sp24 {
 
@@ -439,6 +442,92 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
   return launch_status();
 }
 
+
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
+sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
+                        cudaStream_t s) {
+  using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
+  auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC>;
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    attr_set |= bit;
+  }
+  const int el = kDtype == SP24_BF16 ? 2 : 1;
+  const CUtensorMapDataType dt =
+      kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  // B: each CTA loads BN/2 token rows
+  CUtensorMap mb;
+  SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(g.k), static_cast<uint64_t>(g.m),
+                    static_cast<uint32_t>(128 / el), static_cast<uint32_t>(C::kHalfN)));
+  // E: metadata chunks as rows of 256 bytes (8 rows per 2048-byte chunk)
+  const int64_t kchunks = (g.k + 127) / 128;
+  const int64_t rt128 = (g.n + 127) / 128;
+  CUtensorMap me;
+  SP24_TRY(make_map(&me, g.meta, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 32,
+                    static_cast<uint64_t>(rt128 * kchunks * 8), 32,
+                    static_cast<uint32_t>(8 * C::kMetaChunks), CU_TENSOR_MAP_SWIZZLE_NONE));
+  const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                  : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int y_box = static_cast<int>(g.n < C::kChBox ? g.n : C::kChBox);
+  CUtensorMap my;
+  SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), C::kChunk,
+                    CU_TENSOR_MAP_SWIZZLE_NONE));
+  PersistArgs a;
+  a.meta = g.meta;
+  a.s_x = g.s_x;
+  a.s_w = g.s_w;
+  a.s_y = g.s_y;
+  a.m = g.m;
+  a.n = g.n;
+  a.k = g.k;
+  a.kblocks = g.kblocks;
+  a.row_tiles = static_cast<int>((g.n + 255) / 256);
+  a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
+  const int64_t row_tile_bytes = 256 * (g.k / 2) * el;
+  int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
+  a.group_rows = static_cast<int>(gr);
+  a.y_box = y_box;
+  const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
+  if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
+  const int64_t max_pairs = sm_count() / 2;
+  const int pairs = static_cast<int>(ntiles < max_pairs ? ntiles : max_pairs);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, me, my, a);
+  if (le != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", le);
+  return launch_status();
+}
+
+// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair128 |
+// single (tuning override; default chooses by problem size).
+int impl_choice() {
+  const char* e = std::getenv("SP24_GEMM_IMPL");
+  if (!e) return 0;
+  if (std::strcmp(e, "pair256") == 0) return 1;
+  if (std::strcmp(e, "pair128") == 0) return 2;
+  if (std::strcmp(e, "single") == 0) return 3;
+  return 0;
+}
+
 // Tile plan: BN from the token count, split-K from how many tiles exist.
 template <int kDtype>
 sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s) {
@@ -462,6 +551,29 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
                     box_cols, static_cast<uint32_t>(bn)));
 
   if (split == 1 && bn == 128) {
+    int impl = impl_choice();
+    // pairs pay off once each tile has a long K loop (measured on B200: the
+    // 256 x 256 pair tile wins for K >= 1024 with M, N >= 512; short-K or
+    // narrow-N problems such as K = 768 or N = 64 are faster on single SMs)
+    if (impl == 0) impl = (a.kblocks >= 8 && a.m >= 512 && a.n >= 512) ? 1 : 3;
+    if (impl == 1) {
+      if constexpr (kDtype == SP24_BF16) {
+        return launch_pair<kDtype, 256, 4, SP24_OUT_BF16, 1>(ma, a, x, s);
+      } else {
+        if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, 256, 3, SP24_OUT_INT32, 1>(ma, a, x, s);
+        if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, 256, 4, SP24_OUT_INT8, 1>(ma, a, x, s);
+        return launch_pair<kDtype, 256, 4, SP24_OUT_BF16, 1>(ma, a, x, s);
+      }
+    }
+    if (impl == 2) {
+      if constexpr (kDtype == SP24_BF16) {
+        return launch_pair<kDtype, 128, 6, SP24_OUT_BF16, 2>(ma, a, x, s);
+      } else {
+        if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, 128, 5, SP24_OUT_INT32, 2>(ma, a, x, s);
+        if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, 128, 6, SP24_OUT_INT8, 2>(ma, a, x, s);
+        return launch_pair<kDtype, 128, 5, SP24_OUT_BF16, 2>(ma, a, x, s);
+      }
+    }
     if constexpr (kDtype == SP24_BF16) {
       return launch_persistent<kDtype, 128, 4, SP24_OUT_BF16>(ma, mb, a, s);
     } else {

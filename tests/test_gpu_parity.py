@@ -411,3 +411,44 @@ def test_gemm_int8_full_config_sampled():
     y32, _, _ = _int8_pipeline(w.W, w.X, B.SP24_OUT_INT32)
     assert np.array_equal(y32[torch.from_numpy(rows).cuda()].cpu().numpy(), acc)
     ok_status()
+
+
+# ------------------------------------------------ large-problem kernel variants
+IMPL_SHAPES = [(2500, 2056, 400), (300, 256, 128), (130, 520, 96), (4099, 1032, 784),
+               (200, 64, 128), (3000, 1800, 1296)]
+
+
+@pytest.fixture
+def gemm_impl(request, monkeypatch):
+    monkeypatch.setenv("SP24_GEMM_IMPL", request.param)
+    return request.param
+
+
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair256"], indirect=True)
+@pytest.mark.parametrize("mnk", IMPL_SHAPES)
+def test_gemm_bf16_impls(gemm_impl, mnk):
+    m, n, k = mnk
+    W = I.normal_bf16((n, k), 1.0, seed=41)
+    X = I.normal_bf16((m, k), 1.0, seed=42)
+    _, _, _, y = _bf16_pipeline(W, X)
+    assert_bf16_close(y, *_bf16_ref(W, X))
+    ok_status()
+
+
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair256"], indirect=True)
+@pytest.mark.parametrize("out_kind", [B.SP24_OUT_INT32, B.SP24_OUT_BF16, B.SP24_OUT_INT8])
+@pytest.mark.parametrize("mnk", [(2500, 2064, 416), (130, 528, 96 + 32), (3000, 1808, 1280)])
+def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
+    m, n, k = mnk
+    W = I.long_tail_bf16((n, k), 0.02, seed=51, tail_seed=54)
+    X = I.normal_f32((m, k), 1.0, seed=52)
+    acc, s_x, s_w = _int8_ref(W, X)
+    y, _, _ = _int8_pipeline(W, X, out_kind, s_y=0.05)
+    if out_kind == B.SP24_OUT_INT32:
+        assert np.array_equal(y.cpu().numpy(), acc)
+    elif out_kind == B.SP24_OUT_BF16:
+        got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, O.dequant_bf16(acc, s_x, s_w))
+    else:
+        assert np.array_equal(y.cpu().numpy(), O.requant_int8(acc, s_x, s_w, np.float32(0.05)))
+    ok_status()
