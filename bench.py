@@ -227,14 +227,33 @@ class Runner:
         return t
 
 
-def time_steps(runner, steps, flush, stream):
-    """Per-step CUDA events (L2 flushed before each step, outside the events)."""
+def time_steps(runner, steps, flush, stream, use_graph=True):
+    """Step time: the step captured once in a CUDA graph and replayed, CUDA
+    events around each replay, L2 flushed before each step (outside the
+    events).  Per-stage times: a second pass of plain launches with events
+    between the stages."""
+    tot = []
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            runner.step()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for i in range(steps):
+            flush.zero_()
+            ev[i][0].record()
+            graph.replay()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        tot = [a.elapsed_time(b) for a, b in ev]
+        del graph
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
     for i in range(steps):
         flush.zero_()
         runner.step(evs[i])
     torch.cuda.synchronize()
-    tot = [e[0].elapsed_time(e[3]) for e in evs]
+    if not use_graph:
+        tot = [e[0].elapsed_time(e[3]) for e in evs]
     prune = [e[0].elapsed_time(e[1]) for e in evs]
     comp = [e[1].elapsed_time(e[2]) for e in evs]
     gemm = [e[2].elapsed_time(e[3]) for e in evs]
@@ -351,6 +370,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time plain launches instead of a CUDA-graph replay of the step")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
@@ -389,7 +410,8 @@ def main(argv=None):
 
     barrier()
     with ClockSampler(local) as clk:
-        tot, prune, comp, gemm = time_steps(runner, args.steps, flush, stream)
+        tot, prune, comp, gemm = time_steps(runner, args.steps, flush, stream,
+                                            use_graph=not args.no_graph)
     barrier()
     total_ms = sum(tot)
     if world > 1:
@@ -447,7 +469,8 @@ def main(argv=None):
         "dtype": "int8" if wl.int8 else "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K,
                    "mode": wl.mode, "progressive": wl.progressive,
-                   "l2": "flushed between steps (512 MB write)", "parallelism": f"replicas{world}"},
+                   "l2": "flushed between steps (512 MB write)", "parallelism": f"replicas{world}",
+                   "timing": "plain launches" if args.no_graph else "CUDA graph of one step"},
         "gemm": {"ms": gemm_ms, "tflops_dense_equiv": g_tflops, "gbs": g_gbs,
                  "frac_sparse_peak": g_tflops / sparse_peak},
         "prune_compress": {"ms": comp_ms, "gbs": c_gbs, "frac_hbm": c_gbs / peaks["hbm_gbs"],

@@ -175,15 +175,17 @@ __device__ __forceinline__ uint32_t meta_nibble(uint32_t keep, uint32_t& bad) {
 template <int kDtype>
 struct CompressOut;
 
-// One CTA per metadata chunk (128 rows x 128 K).  256 threads, each takes one
-// 8-weight vector per step (16 vectors per chunk row), so a warp reads two
-// chunk rows of 256 contiguous bytes.  The metadata chunk is assembled in
-// shared memory and written out with 16-byte stores.
+// One CTA per metadata chunk (128 rows x 128 K).  256 threads; thread t owns
+// vector (t % 16) of chunk rows t/16, t/16 + 16, ..., t/16 + 112, i.e. the same
+// 8 K-positions in 8 rows, so a warp reads two chunk rows of 256 contiguous
+// bytes per step.  All 8 loads are issued before any compute (8 x 16 bytes in
+// flight per thread).  The metadata chunk is assembled in shared memory and
+// written out with 16-byte stores.
 //
 // kPrune: compute the keep mask here (magnitude / Wanda, n_keep = 2) instead
 // of reading it; optionally also write it to mask_out.
 template <int kDtype, bool kPrune, bool kWanda>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 3)
 compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask,
                 const uint8_t* __restrict__ mask_in, uint8_t* __restrict__ mask_out,
                 const double* __restrict__ norms, const float* __restrict__ s_w, int64_t n,
@@ -193,34 +195,62 @@ compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask
   const int64_t rt = blockIdx.y;                 // row tile of 128
   const int64_t kblocks = gridDim.x;
   const int64_t kvec = k / 8;
+  const uint32_t bb = threadIdx.x & 15u;         // vector within the chunk row
+  const uint32_t m0 = threadIdx.x >> 4;          // first chunk row (0..15)
+  const int64_t kv = kb * 16 + bb;               // vector index within a row
+  const bool kv_ok = kv < kvec;
   uint32_t bad = 0;
 
+  uint4 q[8];
+  uint32_t keepv[8];
+#pragma unroll
   for (int step = 0; step < 8; ++step) {
-    const uint32_t idx = step * 256u + threadIdx.x;   // 0 .. 2047
-    const uint32_t m = idx >> 4;                      // chunk row
-    const uint32_t bb = idx & 15u;                    // vector within the chunk row
-    const int64_t row = rt * 128 + m;
-    const int64_t kv = kb * 16 + bb;                  // vector index within the row
-    uint32_t meta_byte = 0x44u;                       // padding: positions (0,1)
-    if (row < n && kv < kvec) {
+    const int64_t row = rt * 128 + m0 + 16 * step;
+    keepv[step] = 0xFFu;
+    if (row < n && kv_ok) {
       const int64_t vi = row * kvec + kv;
-      const uint4 q = __ldcs(reinterpret_cast<const uint4*>(w) + vi);
+      q[step] = __ldcs(reinterpret_cast<const uint4*>(w) + vi);
+      if constexpr (kPrune) {
+        if (mask_in) keepv[step] = mask_in[vi];
+      } else {
+        keepv[step] = mask[vi];
+      }
+    }
+  }
+  double nrm[8];
+  if constexpr (kPrune && kWanda) {
+    if (kv_ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + kv * 8 + i);
+    }
+  }
+  float s_row[8];
+  if constexpr (kDtype == SP24_INT8) {
+#pragma unroll
+    for (int step = 0; step < 8; ++step) {
+      const int64_t row = rt * 128 + m0 + 16 * step;
+      s_row[step] = row < n ? s_w[row] : 1.0f;
+    }
+  }
+
+#pragma unroll
+  for (int step = 0; step < 8; ++step) {
+    const uint32_t m = m0 + 16 * step;
+    const int64_t row = rt * 128 + m;
+    uint32_t meta_byte = 0x44u;                  // padding: positions (0,1)
+    if (row < n && kv_ok) {
+      const int64_t vi = row * kvec + kv;
       uint32_t keep;
       if constexpr (kPrune) {
-        double nrm[8];
-        if constexpr (kWanda) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + kv * 8 + i);
-        }
-        keep = mask_byte<kWanda>(q, mask_in ? mask_in[vi] : 0xFFu, nrm, 2);
+        keep = mask_byte<kWanda>(q[step], keepv[step], nrm, 2);
         if (mask_out) mask_out[vi] = static_cast<uint8_t>(keep);
       } else {
-        keep = mask[vi];
+        keep = keepv[step];
       }
       const uint32_t n0 = meta_nibble(keep & 15u, bad);
       const uint32_t n1 = meta_nibble(keep >> 4, bad);
       meta_byte = n0 | (n1 << 4);
-      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+      const uint32_t words[4] = {q[step].x, q[step].y, q[step].z, q[step].w};
       uint32_t sel[4];
       const uint32_t pos[4] = {n0 & 3u, n0 >> 2, 4u + (n1 & 3u), 4u + (n1 >> 2)};
 #pragma unroll
@@ -232,18 +262,17 @@ compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask
         uint2 o;
         o.x = sel[0] | (sel[1] << 16);
         o.y = sel[2] | (sel[3] << 16);
-        reinterpret_cast<uint2*>(vals)[vi] = o;
+        __stcs(reinterpret_cast<uint2*>(vals) + vi, o);
       } else {
-        const float s = s_w[row];
         uint32_t packed = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float x = __uint_as_float(sel[i] << 16);
-          int qv = __float2int_rn(__fdiv_rn(x, s));
+          int qv = __float2int_rn(__fdiv_rn(x, s_row[step]));
           qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
           packed |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * i);
         }
-        reinterpret_cast<uint32_t*>(vals)[vi] = packed;
+        __stcs(reinterpret_cast<unsigned int*>(vals) + vi, packed);
       }
     }
     chunk[meta_offset<kDtype>(m, bb)] = static_cast<uint8_t>(meta_byte);
@@ -252,7 +281,7 @@ compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask
   __syncthreads();
   if (threadIdx.x < 128) {
     uint4* dst = reinterpret_cast<uint4*>(meta + (rt * kblocks + kb) * 2048);
-    dst[threadIdx.x] = reinterpret_cast<const uint4*>(chunk)[threadIdx.x];
+    __stcs(dst + threadIdx.x, reinterpret_cast<const uint4*>(chunk)[threadIdx.x]);
   }
 }
 
