@@ -203,6 +203,35 @@ sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
                       const float* s_w, int out_kind, const float* s_y, void* Y,
                       void* stream);
 
+/* ------------------------------------------------- allocation-free variant */
+
+/* Largest K accepted by sp24_prune_wanda_noalloc. */
+#define SP24_NOALLOC_MAX_K 65536
+
+/* Wanda pruning for callers that cannot allocate device memory.  It computes
+ * exactly what sp24_prune(W, N, K, Xc, Mc, SP24_WANDA, n_keep, mask_in,
+ * mask_out, workspace, stream) computes, but keeps the float64 column norms in
+ * a scratch array inside the library instead of a caller workspace, so the
+ * caller passes only inputs and outputs.  Meant for code that must not call
+ * cudaMalloc: inference engines and plugins whose device memory plan is fixed
+ * at start-up, and code that runs where allocation would synchronise the
+ * device or is not permitted.  (The pages have no counterpart; this is an
+ * interface convenience.)
+ *   - The scratch array holds SP24_NOALLOC_MAX_K doubles (512 KiB); every GPU
+ *     that loads the library keeps it until the process exits.  K larger than
+ *     SP24_NOALLOC_MAX_K returns SP24_ERR_UNSUPPORTED before any launch.
+ *   - The first call on a device looks up the array's device address (a
+ *     one-time set-up per device); make that first call before any stream
+ *     capture on the device.
+ *   - All calls share the one array and each call overwrites all K entries it
+ *     uses before reading them.  Calls that overlap on the GPU (for example on
+ *     two streams at once) race on it and must be serialised by the caller.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Arguments, rules and errors are those of sp24_prune with mode SP24_WANDA. */
+sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const void* Xc,
+                                     int64_t Mc, int n_keep, const uint8_t* mask_in,
+                                     uint8_t* mask_out, void* stream);
+
 /* --------------------------------------------------------------- status */
 
 /* Synchronises `stream`, then returns and clears the device status word of the

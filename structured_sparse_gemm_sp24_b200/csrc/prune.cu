@@ -11,6 +11,8 @@
 // [Ampere-sparsity] NVIDIA x Tencent article, Figure 1 (values + index
 // metadata), Figure 4 (progressive 25 % -> 50 %), "PTQ and QAT" (99.99 %
 // coverage scale).
+#include <mutex>
+
 #include "sp24_device.cuh"
 #include "sp24_host.h"
 
@@ -465,6 +467,39 @@ __global__ void quantize_tail(const float* __restrict__ x, int64_t start, int64_
   if (i < count) xq[i] = static_cast<int8_t>(q8(x[i], *s_ptr));
 }
 
+
+// ------------------------------------------- Wanda prune without allocation
+// For callers that may not allocate device memory (see sp24_prune_wanda_noalloc
+// in include/sp24.h): the float64 column norms live in this file-scope array
+// instead of a caller workspace.  Every GPU that loads the library holds it
+// (SP24_NOALLOC_MAX_K * 8 bytes) until the process exits.
+__device__ __align__(256) double g_noalloc_norms[SP24_NOALLOC_MAX_K];
+
+namespace {
+constexpr int kNoallocMaxDevices = 64;
+double* g_noalloc_ptr[kNoallocMaxDevices];   // device address of the array, per device
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_norms on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+sp24_status noalloc_norms(double** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  if (dev < 0 || dev >= kNoallocMaxDevices) return SP24_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_norms);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress", e);
+    g_noalloc_ptr[dev] = static_cast<double*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return SP24_OK;
+}
+}  // namespace
+
 // -------------------------------------------------------------- launching
 static int grid_for(int64_t work_items, int threads) {
   const int64_t want = (work_items + threads - 1) / threads;
@@ -528,6 +563,27 @@ sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc, int6
     prune_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W), nvec, K / 8, nullptr,
                                              mask_in, mask_out, n_keep);
   }
+  return launch_status();
+}
+
+sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const void* Xc,
+                                     int64_t Mc, int n_keep, const uint8_t* mask_in,
+                                     uint8_t* mask_out, void* stream) {
+  if (N < 0 || K < 0 || (n_keep != 2 && n_keep != 3)) return SP24_ERR_ARG;
+  if (K > SP24_NOALLOC_MAX_K) return SP24_ERR_UNSUPPORTED;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!W || !mask_out || !Xc || Mc < 1) return SP24_ERR_ARG;
+  if (K % 8 != 0 || !aligned16(W) || !aligned16(mask_out) || !aligned16(Xc) ||
+      (mask_in && !aligned16(mask_in)))
+    return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  double* norms = nullptr;
+  SP24_TRY(noalloc_norms(&norms));
+  cudaStream_t s = as_stream(stream);
+  SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
+  const int64_t nvec = N * (K / 8);
+  prune_kernel<true><<<grid_for((nvec + 3) / 4, 256), 256, 0, s>>>(
+      static_cast<const uint4*>(W), nvec, K / 8, norms, mask_in, mask_out, n_keep);
   return launch_status();
 }
 

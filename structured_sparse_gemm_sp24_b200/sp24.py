@@ -32,6 +32,7 @@ SP24_INT8 = 1
 SP24_OUT_BF16 = 0
 SP24_OUT_INT32 = 1
 SP24_OUT_INT8 = 2
+SP24_NOALLOC_MAX_K = 65536
 
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
@@ -61,6 +62,8 @@ SIGNATURES = {
     "sp24_strerror": (ctypes.c_char_p, [_c_int]),
     "sp24_version": (_c_int, []),
     "sp24_last_cuda_error": (ctypes.c_char_p, []),
+    "sp24_prune_wanda_noalloc": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_int, _c_p, _c_p,
+                                          _c_p]),
 }
 
 _LIB: Optional[ctypes.CDLL] = None
@@ -157,6 +160,15 @@ def sp24_prune(W: torch.Tensor, Xc: Optional[torch.Tensor], mode: int, n_keep: i
     Mc = 0 if Xc is None else Xc.shape[0]
     _check(lib().sp24_prune(_ptr(W), N, K, _ptr(Xc), Mc, mode, n_keep, _ptr(mask_in),
                             _ptr(mask_out), _ptr(workspace), _stream(stream)), "sp24_prune")
+
+
+def sp24_prune_wanda_noalloc(W: torch.Tensor, Xc: torch.Tensor, n_keep: int,
+                             mask_in: Optional[torch.Tensor], mask_out: torch.Tensor,
+                             stream=None) -> None:
+    N, K = W.shape
+    _check(lib().sp24_prune_wanda_noalloc(_ptr(W), N, K, _ptr(Xc), Xc.shape[0], n_keep,
+                                          _ptr(mask_in), _ptr(mask_out), _stream(stream)),
+           "sp24_prune_wanda_noalloc")
 
 
 def sp24_wscale(W: torch.Tensor, mask: torch.Tensor, coverage: float, s_w: torch.Tensor,
