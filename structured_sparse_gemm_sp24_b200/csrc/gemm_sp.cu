@@ -37,6 +37,7 @@
 
 #include "sp24_device.cuh"
 #include "sp24_host.h"
+#include "tma_host.h"
 
 namespace sp24 {
 
@@ -322,42 +323,6 @@ namespace sp24 {
 
 // ----------------------------------------------------------------- host side
 namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool get_encoder() {
-  std::call_once(g_encode_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  });
-  return g_encode != nullptr;
-}
-
-// 2D row-major [rows][cols] map with a {box_cols, box_rows} box, 128B swizzle,
-// zero fill outside the tensor.
-sp24_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elsize,
-              uint64_t cols, uint64_t rows, uint32_t box_cols, uint32_t box_rows,
-              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elsize)};
-  cuuint32_t box[2] = {box_cols, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  const CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                             CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r == CUDA_SUCCESS) return SP24_OK;
-  char buf[96];
-  std::snprintf(buf, sizeof(buf), "CUresult %d (box %ux%u, dims %llux%llu)", static_cast<int>(r),
-                box_cols, box_rows, static_cast<unsigned long long>(cols),
-                static_cast<unsigned long long>(rows));
-  return cuda_fail("cuTensorMapEncodeTiled", buf);
-}
 
 template <int kDtype, int BN, int STAGES, int SPLIT>
 sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& a,

@@ -15,6 +15,7 @@
 
 #include "sp24_device.cuh"
 #include "sp24_host.h"
+#include "tma_host.h"
 
 namespace sp24 {
 
@@ -75,6 +76,73 @@ __device__ __forceinline__ uint32_t mask_byte(const uint4& w, uint32_t in, const
   return out;
 }
 
+// ------------------------------------------------ fast magnitude selection
+// Augmented keys K_p = (|w_p| bits << 2) | (3 - p) of one group (4 bf16 in two
+// 32-bit words): all distinct, and K_q > K_p exactly when q beats p under the
+// rank rule (larger magnitude; equal magnitudes go to the lower index).  A
+// position dropped by mask_in scores magnitude 0 and keeps its index order.
+// The kept set is then the n_keep largest keys.
+template <bool kLive>
+__device__ __forceinline__ uint32_t keep_nibble_mag(uint32_t w0, uint32_t w1, uint32_t live,
+                                                    int n_keep) {
+  uint32_t k0 = ((w0 << 2) & 0x1FFFCu) | 3u;
+  uint32_t k1 = ((w0 >> 14) & 0x1FFFCu) | 2u;
+  uint32_t k2 = ((w1 << 2) & 0x1FFFCu) | 1u;
+  uint32_t k3 = ((w1 >> 14) & 0x1FFFCu);
+  if constexpr (kLive) {
+    k0 = (live & 1u) ? k0 : 3u;
+    k1 = (live & 2u) ? k1 : 2u;
+    k2 = (live & 4u) ? k2 : 1u;
+    k3 = (live & 8u) ? k3 : 0u;
+  }
+  const uint32_t a = max(k0, k1), b = min(k0, k1), c = max(k2, k3), d = min(k2, k3);
+  if (n_keep == 2) {
+    const uint32_t t1 = max(a, c);
+    const uint32_t t2 = max(min(a, c), max(b, d));
+    return (1u << (~t1 & 3u)) | (1u << (~t2 & 3u));
+  }
+  const uint32_t t4 = min(b, d);   // n_keep == 3: drop the smallest
+  return 0xFu ^ (1u << (~t4 & 3u));
+}
+
+// Positions (lo < hi) of the two largest augmented keys of a group (see
+// keep_nibble_mag), with integer min/max only.
+template <bool kLive>
+__device__ __forceinline__ void top2_positions_mag(uint32_t w0, uint32_t w1, uint32_t live,
+                                                   uint32_t& lo, uint32_t& hi) {
+  uint32_t k0 = ((w0 << 2) & 0x1FFFCu) | 3u;
+  uint32_t k1 = ((w0 >> 14) & 0x1FFFCu) | 2u;
+  uint32_t k2 = ((w1 << 2) & 0x1FFFCu) | 1u;
+  uint32_t k3 = ((w1 >> 14) & 0x1FFFCu);
+  if constexpr (kLive) {
+    k0 = (live & 1u) ? k0 : 3u;
+    k1 = (live & 2u) ? k1 : 2u;
+    k2 = (live & 4u) ? k2 : 1u;
+    k3 = (live & 8u) ? k3 : 0u;
+  }
+  const uint32_t a = max(k0, k1), b = min(k0, k1), c = max(k2, k3), d = min(k2, k3);
+  const uint32_t p1 = ~max(a, c) & 3u;                     // 3 - (t & 3)
+  const uint32_t p2 = ~max(min(a, c), max(b, d)) & 3u;
+  lo = min(p1, p2);
+  hi = max(p1, p2);
+}
+
+// Metadata code (lo | hi << 2) of a keep nibble from a 16-entry table; nibbles
+// without exactly two bits set map to positions (0, 1) and are flagged.
+constexpr uint64_t kNibbleCode = 0x444E4DC449844444ull;   // indices 3,5,6,9,10,12 valid
+constexpr uint32_t kNibbleValid = 0x1668u;
+__device__ __forceinline__ uint32_t nibble_code(uint32_t nib, uint32_t& bad) {
+  bad |= ((kNibbleValid >> nib) & 1u) ^ 1u;
+  return static_cast<uint32_t>(kNibbleCode >> (4u * nib)) & 0xFu;
+}
+
+// Gathers the kept bf16 pair of a group with one byte permute: low half =
+// position lo, high half = position hi.
+__device__ __forceinline__ uint32_t gather_pair(uint32_t w0, uint32_t w1, uint32_t lo,
+                                                uint32_t hi) {
+  return __byte_perm(w0, w1, 0x1010u + 0x22u * lo + 0x2200u * hi);
+}
+
 // -------------------------------------------------------------- a1 colnorm
 // Block per 64 columns.  Each pass stages a [128 tokens][64 columns] bf16 tile
 // in shared memory with every 16-byte load in flight, then threads 0..63 add
@@ -105,43 +173,6 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const uint16_t* __restrict
     __syncthreads();
   }
   if (threadIdx.x < cvalid) norms[col0 + threadIdx.x] = __dsqrt_rn(acc);
-}
-
-// ------------------------------------------------------------ a2+a3 prune
-// Flat over W: vector v = 8 consecutive weights = one mask byte (K % 8 == 0,
-// so a vector never straddles two rows).  Grid-stride, 4 vectors in flight.
-template <bool kWanda>
-__global__ void __launch_bounds__(256) prune_kernel(const uint4* __restrict__ w, int64_t nvec,
-                                                    int64_t kvec, const double* __restrict__ norms,
-                                                    const uint8_t* __restrict__ mask_in,
-                                                    uint8_t* __restrict__ mask_out, int n_keep) {
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (; v < nvec; v += 4 * stride) {
-    uint4 q[4];
-    uint32_t in[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t vu = v + u * stride;
-      if (vu < nvec) {
-        q[u] = __ldcs(w + vu);
-        in[u] = mask_in ? mask_in[vu] : 0xFFu;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int64_t vu = v + u * stride;
-      if (vu < nvec) {
-        double nrm[8];
-        if constexpr (kWanda) {
-          const int64_t col = (vu % kvec) * 8;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + col + i);
-        }
-        mask_out[vu] = static_cast<uint8_t>(mask_byte<kWanda>(q[u], in[u], nrm, n_keep));
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------ a4 compress
@@ -177,114 +208,205 @@ __device__ __forceinline__ uint32_t meta_nibble(uint32_t keep, uint32_t& bad) {
 template <int kDtype>
 struct CompressOut;
 
-// One CTA per metadata chunk (128 rows x 128 K).  256 threads; thread t owns
-// vector (t % 16) of chunk rows t/16, t/16 + 16, ..., t/16 + 112, i.e. the same
-// 8 K-positions in 8 rows, so a warp reads two chunk rows of 256 contiguous
-// bytes per step.  All 8 loads are issued before any compute (8 x 16 bytes in
-// flight per thread).  The metadata chunk is assembled in shared memory and
-// written out with 16-byte stores.
-//
-// kPrune: compute the keep mask here (magnitude / Wanda, n_keep = 2) instead
-// of reading it; optionally also write it to mask_out.
-template <int kDtype, bool kPrune, bool kWanda>
-__global__ void __launch_bounds__(256, 3)
-compress_kernel(const uint16_t* __restrict__ w, const uint8_t* __restrict__ mask,
-                const uint8_t* __restrict__ mask_in, uint8_t* __restrict__ mask_out,
-                const double* __restrict__ norms, const float* __restrict__ s_w, int64_t n,
-                int64_t k, void* __restrict__ vals, uint8_t* __restrict__ meta) {
-  __shared__ __align__(16) uint8_t chunk[2048];
-  const int64_t kb = blockIdx.x;                 // K block of 128
-  const int64_t rt = blockIdx.y;                 // row tile of 128
-  const int64_t kblocks = gridDim.x;
-  const int64_t kvec = k / 8;
-  const uint32_t bb = threadIdx.x & 15u;         // vector within the chunk row
-  const uint32_t m0 = threadIdx.x >> 4;          // first chunk row (0..15)
-  const int64_t kv = kb * 16 + bb;               // vector index within a row
-  const bool kv_ok = kv < kvec;
+// ------------------------------------------- a2..a4 streaming chunk kernel
+// One persistent CTA per SM walks 128-row x 128-K chunks of W.  Thread 0
+// keeps kStreamStages chunks in flight with TMA loads (the W chunk plus, as
+// needed, the chunk's mask bytes, the 128 Wanda column norms and the 128
+// per-row INT8 scales); the 1024 threads then work from shared memory: thread
+// t takes vector t % 16 (8 consecutive K-positions) of chunk rows t/16 + 64*j,
+// j = 0..1, so a warp reads two rows of 256 contiguous bytes.
+//   kPrune: compute the keep mask (magnitude / Wanda, n_keep of 4) from W,
+//           with dropped mask_in positions scoring 0; else read the mask.
+//   kVals:  kValsNone   -> write the keep mask only (sp24_prune);
+//           kValsBF16/INT8 -> also write values and the metadata chunk.
+// The metadata chunk and the mask bytes of a chunk are assembled in shared
+// memory and written with 16-byte stores.
+enum { kValsNone = 0, kValsBF16 = 1, kValsINT8 = 2 };
+
+constexpr int kStreamStages = 5;
+constexpr int kStreamThreads = 1024;
+constexpr int kWTile = 128 * 256;          // 128 rows x 128 bf16
+constexpr int kMTile = 128 * 16;           // 128 rows x 16 mask bytes
+constexpr int kNTile = 128 * 8;            // 128 float64 norms
+constexpr int kSTile = 128 * 4;            // 128 float32 row scales
+constexpr int kStreamStage = kWTile + kMTile + kNTile + kSTile;   // multiple of 128
+constexpr int kStreamSmem = kStreamStages * kStreamStage + 4 * 2048 + 256 + 1024;
+
+struct StreamArgs {
+  int64_t n, k;
+  int kblocks;                 // chunks along K
+  int nchunks;                 // row tiles * kblocks
+  int n_keep;
+  int mask_tma;                // the chunk's mask bytes come with the TMA stage
+  const uint8_t* mask_direct;  // else read from here (NULL: no mask / mask_in)
+  uint8_t* mask_out;           // NULL: not written
+  void* vals;
+  uint8_t* meta;
+};
+
+template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_mask,
+              const __grid_constant__ CUtensorMap tm_norm, const __grid_constant__ CUtensorMap tm_sw,
+              const StreamArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* meta_buf = smem + kStreamStages * kStreamStage;     // 2 x 2048
+  uint8_t* mout_buf = meta_buf + 2 * 2048;                     // 2 x 2048
+  uint64_t* full = reinterpret_cast<uint64_t*>(mout_buf + 2 * 2048);
+
+  const int tid = threadIdx.x;
+  const uint32_t bb = tid & 15u;              // vector within a chunk row
+  const uint32_t m0 = tid >> 4;               // first chunk row (0..63)
+  const int64_t kvec = a.k / 8;
+  const int nmine = a.nchunks > static_cast<int>(blockIdx.x)
+                        ? (a.nchunks - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
+                        : 0;
+  const bool use_mask_tile = a.mask_tma != 0;
+  const uint32_t stage_tx = kWTile + (use_mask_tile ? kMTile : 0) + (kWanda ? kNTile : 0) +
+                            (kVals == kValsINT8 ? kSTile : 0);
+
+  if (tid == 0) {
+    for (int st = 0; st < kStreamStages; ++st) mbar_init(&full[st], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto issue = [&](int i) {
+    const int c = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    const int rt = c / a.kblocks, kb = c - rt * a.kblocks;
+    const int st = i % kStreamStages;
+    uint8_t* sb = smem + st * kStreamStage;
+    mbar_arrive_expect_tx(&full[st], stage_tx);
+    tma_load_2d(sb, &tm_w, &full[st], kb * 128, rt * 128);
+    if (use_mask_tile) tma_load_2d(sb + kWTile, &tm_mask, &full[st], kb * 16, rt * 128);
+    if constexpr (kWanda) tma_load_1d(sb + kWTile + kMTile, &tm_norm, &full[st], kb * 128);
+    if constexpr (kVals == kValsINT8)
+      tma_load_1d(sb + kWTile + kMTile + kNTile, &tm_sw, &full[st], rt * 128);
+  };
+  if (tid == 0) {
+    prefetch_tmap(&tm_w);
+    for (int i = 0; i < nmine && i < kStreamStages; ++i) issue(i);
+  }
+
   uint32_t bad = 0;
-
-  uint4 q[8];
-  uint32_t keepv[8];
+  for (int i = 0; i < nmine; ++i) {
+    const int c = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    const int rt = c / a.kblocks, kb = c - rt * a.kblocks;
+    const int st = i % kStreamStages;
+    const uint8_t* sb = smem + st * kStreamStage;
+    const bool ready = mbar_wait(&full[st], (i / kStreamStages) & 1u);
+    const int64_t kv = static_cast<int64_t>(kb) * 16 + bb;
+    const bool kv_ok = kv < kvec && ready;
+    uint8_t* mb = meta_buf + (i & 1) * 2048;
+    uint8_t* ob = mout_buf + (i & 1) * 2048;
+    double nrm[8];
+    if constexpr (kWanda) {
 #pragma unroll
-  for (int step = 0; step < 8; ++step) {
-    const int64_t row = rt * 128 + m0 + 16 * step;
-    keepv[step] = 0xFFu;
-    if (row < n && kv_ok) {
-      const int64_t vi = row * kvec + kv;
-      q[step] = __ldcs(reinterpret_cast<const uint4*>(w) + vi);
-      if constexpr (kPrune) {
-        if (mask_in) keepv[step] = mask_in[vi];
-      } else {
-        keepv[step] = mask[vi];
-      }
+      for (int e = 0; e < 8; ++e)
+        nrm[e] = reinterpret_cast<const double*>(sb + kWTile + kMTile)[bb * 8 + e];
     }
-  }
-  double nrm[8];
-  if constexpr (kPrune && kWanda) {
-    if (kv_ok) {
+    // per-thread bases: chunk row m0 + 64 j is +16384 bytes of the W tile,
+    // +1024 bytes of the mask tile, of the metadata chunk (both layouts) and
+    // of the mask staging, and +64 j * kvec vectors in global memory
+    const uint8_t* wrow = sb + m0 * 256 + bb * 16;
+    const uint8_t* mrow = sb + kWTile + m0 * 16 + bb;
+    const float* srow = reinterpret_cast<const float*>(sb + kWTile + kMTile + kNTile) + m0;
+    const uint32_t moff = kVals == kValsINT8 ? meta_offset<SP24_INT8>(m0, bb)
+                                             : meta_offset<SP24_BF16>(m0, bb);
+    const int64_t row0 = static_cast<int64_t>(rt) * 128 + m0;
+    const int64_t vi0 = row0 * kvec + kv;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) nrm[i] = __ldg(norms + kv * 8 + i);
-    }
-  }
-  float s_row[8];
-  if constexpr (kDtype == SP24_INT8) {
-#pragma unroll
-    for (int step = 0; step < 8; ++step) {
-      const int64_t row = rt * 128 + m0 + 16 * step;
-      s_row[step] = row < n ? s_w[row] : 1.0f;
-    }
-  }
-
-#pragma unroll
-  for (int step = 0; step < 8; ++step) {
-    const uint32_t m = m0 + 16 * step;
-    const int64_t row = rt * 128 + m;
-    uint32_t meta_byte = 0x44u;                  // padding: positions (0,1)
-    if (row < n && kv_ok) {
-      const int64_t vi = row * kvec + kv;
-      uint32_t keep;
-      if constexpr (kPrune) {
-        keep = mask_byte<kWanda>(q[step], keepv[step], nrm, 2);
-        if (mask_out) mask_out[vi] = static_cast<uint8_t>(keep);
-      } else {
-        keep = keepv[step];
-      }
-      const uint32_t n0 = meta_nibble(keep & 15u, bad);
-      const uint32_t n1 = meta_nibble(keep >> 4, bad);
-      meta_byte = n0 | (n1 << 4);
-      const uint32_t words[4] = {q[step].x, q[step].y, q[step].z, q[step].w};
-      uint32_t sel[4];
-      const uint32_t pos[4] = {n0 & 3u, n0 >> 2, 4u + (n1 & 3u), 4u + (n1 >> 2)};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t word = words[pos[i] >> 1];
-        sel[i] = (pos[i] & 1u) ? (word >> 16) : (word & 0xFFFFu);
-      }
-      if constexpr (kDtype == SP24_BF16) {
-        uint2 o;
-        o.x = sel[0] | (sel[1] << 16);
-        o.y = sel[2] | (sel[3] << 16);
-        __stcs(reinterpret_cast<uint2*>(vals) + vi, o);
-      } else {
-        uint32_t packed = 0;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float x = __uint_as_float(sel[i] << 16);
-          int qv = __float2int_rn(__fdiv_rn(x, s_row[step]));
-          qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
-          packed |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * i);
+    for (int j = 0; j < 2; ++j) {
+      const bool ok = kv_ok && row0 + 64 * j < a.n;
+      const int64_t vi = vi0 + static_cast<int64_t>(64 * j) * kvec;
+      uint32_t meta_byte = 0x44u;             // padding: positions (0, 1)
+      uint32_t keep = 0;
+      if (ok) {
+        const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16384 * j);
+        uint32_t mbyte = 0xFFu;
+        if (!kPrune || kMaskIn) {
+          if (use_mask_tile) {
+            mbyte = mrow[1024 * j];
+          } else {
+            mbyte = a.mask_direct[vi];
+          }
         }
-        __stcs(reinterpret_cast<unsigned int*>(vals) + vi, packed);
+        uint32_t lo0, hi0, lo1, hi1;
+        if constexpr (kPrune && !kWanda && kVals != kValsNone) {
+          top2_positions_mag<kMaskIn>(q.x, q.y, mbyte & 15u, lo0, hi0);
+          top2_positions_mag<kMaskIn>(q.z, q.w, mbyte >> 4, lo1, hi1);
+          if (a.mask_out) keep = (1u << lo0) | (1u << hi0) | (((1u << lo1) | (1u << hi1)) << 4);
+        } else {
+          if constexpr (kPrune && kWanda) {
+            keep = mask_byte<true>(q, mbyte, nrm, a.n_keep);
+          } else if constexpr (kPrune) {
+            keep = keep_nibble_mag<kMaskIn>(q.x, q.y, mbyte & 15u, a.n_keep) |
+                   (keep_nibble_mag<kMaskIn>(q.z, q.w, mbyte >> 4, a.n_keep) << 4);
+          } else {
+            keep = mbyte;
+          }
+          if constexpr (kVals != kValsNone) {
+            uint32_t badv = 0;
+            const uint32_t c0 = nibble_code(keep & 15u, badv);
+            const uint32_t c1 = nibble_code(keep >> 4, badv);
+            if (!kPrune) bad |= badv;
+            lo0 = c0 & 3u; hi0 = c0 >> 2; lo1 = c1 & 3u; hi1 = c1 >> 2;
+          }
+        }
+        if constexpr (kVals != kValsNone) {
+          meta_byte = lo0 | (hi0 << 2) | (lo1 << 4) | (hi1 << 6);
+          const uint32_t p0 = gather_pair(q.x, q.y, lo0, hi0);
+          const uint32_t p1 = gather_pair(q.z, q.w, lo1, hi1);
+          if constexpr (kVals == kValsBF16) {
+            __stcs(reinterpret_cast<uint2*>(a.vals) + vi, make_uint2(p0, p1));
+          } else {
+            const float sc = srow[64 * j];
+            const float xs[4] = {__uint_as_float(p0 << 16), __uint_as_float(p0 & 0xFFFF0000u),
+                                 __uint_as_float(p1 << 16), __uint_as_float(p1 & 0xFFFF0000u)};
+            uint32_t packed = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              int qv = __float2int_rn(__fdiv_rn(xs[e], sc));
+              qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
+              packed |= (static_cast<uint32_t>(qv) & 0xFFu) << (8 * e);
+            }
+            __stcs(reinterpret_cast<unsigned int*>(a.vals) + vi, packed);
+          }
+        }
+      }
+      if constexpr (kVals != kValsNone) mb[moff + 1024 * j] = meta_byte;
+      if (a.mask_out) ob[m0 * 16 + bb + 1024 * j] = static_cast<uint8_t>(keep);
+    }
+    __syncthreads();   // stage `st` fully read; chunk buffers complete
+    if (tid == 0 && i + kStreamStages < nmine) {
+      fence_async_shared();
+      issue(i + kStreamStages);
+    }
+    if constexpr (kVals != kValsNone) {
+      if (tid < 128) {
+        uint4* dst = reinterpret_cast<uint4*>(
+            a.meta + (static_cast<int64_t>(rt) * a.kblocks + kb) * 2048);
+        __stcs(dst + tid, reinterpret_cast<const uint4*>(mb)[tid]);
       }
     }
-    chunk[meta_offset<kDtype>(m, bb)] = static_cast<uint8_t>(meta_byte);
+    if (a.mask_out && tid >= 256 && tid < 384) {
+      const int m = tid - 256;
+      const int64_t row = static_cast<int64_t>(rt) * 128 + m;
+      const int64_t v0 = static_cast<int64_t>(kb) * 16;
+      int nb = static_cast<int>(kvec - v0 < 16 ? kvec - v0 : 16);
+      if (row < a.n && nb > 0) {
+        uint8_t* dst = a.mask_out + row * kvec + v0;
+        if (nb == 16 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob + m * 16);
+        } else {
+          for (int e = 0; e < nb; ++e) dst[e] = ob[m * 16 + e];
+        }
+      }
+    }
   }
   if (bad) raise_error(kErrPatternBit);
-  __syncthreads();
-  if (threadIdx.x < 128) {
-    uint4* dst = reinterpret_cast<uint4*>(meta + (rt * kblocks + kb) * 2048);
-    __stcs(dst + threadIdx.x, reinterpret_cast<const uint4*>(chunk)[threadIdx.x]);
-  }
 }
 
 // --------------------------------------------------------- a5 weight scale
@@ -514,15 +636,68 @@ static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double*
   return launch_status();
 }
 
-template <int kDtype, bool kPrune, bool kWanda>
-static sp24_status launch_compress(const void* w, const uint8_t* mask, const uint8_t* mask_in,
-                                   uint8_t* mask_out, const double* norms, const float* s_w,
-                                   int64_t n, int64_t k, void* vals, void* meta, cudaStream_t s) {
-  const dim3 grid(static_cast<unsigned>((k + 127) / 128), static_cast<unsigned>((n + 127) / 128));
-  compress_kernel<kDtype, kPrune, kWanda><<<grid, 256, 0, s>>>(
-      static_cast<const uint16_t*>(w), mask, mask_in, mask_out, norms, s_w, n, k, vals,
-      static_cast<uint8_t*>(meta));
+template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
+static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* mask_out,
+                                 const double* norms, const float* s_w, int64_t n, int64_t k,
+                                 int n_keep, void* vals, void* meta, cudaStream_t s) {
+  auto kern = stream_kernel<kPrune, kWanda, kVals, kMaskIn>;
+  static uint64_t attr_set = 0;   // one bit per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    attr_set |= bit;
+  }
+  const int64_t kblocks = (k + 127) / 128;
+  const int64_t nchunks = ((n + 127) / 128) * kblocks;
+  if (nchunks > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
+  CUtensorMap tw, tm, tn, ts;
+  SP24_TRY(make_map(&tw, w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, static_cast<uint64_t>(k),
+                    static_cast<uint64_t>(n), 128, 128, CU_TENSOR_MAP_SWIZZLE_NONE));
+  // mask bytes ride along with the TMA stage when their rows are 16-byte aligned
+  const bool mask_tma = mask != nullptr && (k % 128) == 0;
+  tm = tw;
+  if (mask_tma)
+    SP24_TRY(make_map(&tm, mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(k / 8),
+                      static_cast<uint64_t>(n), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE));
+  tn = tw;
+  if (kWanda)
+    SP24_TRY(make_map_1d(&tn, norms, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, static_cast<uint64_t>(k),
+                         128));
+  ts = tw;
+  if (kVals == kValsINT8)
+    SP24_TRY(make_map_1d(&ts, s_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, static_cast<uint64_t>(n),
+                         128));
+  StreamArgs a;
+  a.n = n;
+  a.k = k;
+  a.kblocks = static_cast<int>(kblocks);
+  a.nchunks = static_cast<int>(nchunks);
+  a.n_keep = n_keep;
+  a.mask_tma = mask_tma ? 1 : 0;
+  a.mask_direct = mask_tma ? nullptr : mask;
+  a.mask_out = mask_out;
+  a.vals = vals;
+  a.meta = static_cast<uint8_t*>(meta);
+  const int grid = static_cast<int>(nchunks < sm_count() ? nchunks : sm_count());
+  kern<<<grid, kStreamThreads, kStreamSmem, s>>>(tw, tm, tn, ts, a);
   return launch_status();
+}
+
+// For the pruning variants `mask` is mask_in (optional); a separate
+// instantiation without it drops the liveness selects from the inner loop.
+template <bool kPrune, bool kWanda, int kVals>
+static sp24_status launch_stream(const void* w, const uint8_t* mask, uint8_t* mask_out,
+                                 const double* norms, const float* s_w, int64_t n, int64_t k,
+                                 int n_keep, void* vals, void* meta, cudaStream_t s) {
+  if (kPrune && mask == nullptr)
+    return launch_stream_t<kPrune, kWanda, kVals, false>(w, mask, mask_out, norms, s_w, n, k,
+                                                         n_keep, vals, meta, s);
+  return launch_stream_t<kPrune, kWanda, kVals, true>(w, mask, mask_out, norms, s_w, n, k, n_keep,
+                                                      vals, meta, s);
 }
 
 }  // namespace sp24
@@ -552,18 +727,14 @@ sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc, int6
   if (mode == SP24_WANDA && (!aligned16(Xc) || !aligned16(workspace))) return SP24_ERR_ALIGN;
   SP24_TRY(check_device());
   cudaStream_t s = as_stream(stream);
-  const int64_t nvec = N * (K / 8);
-  const int grid = grid_for((nvec + 3) / 4, 256);
   if (mode == SP24_WANDA) {
     double* norms = static_cast<double*>(workspace);
     SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
-    prune_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W), nvec, K / 8, norms,
-                                            mask_in, mask_out, n_keep);
-  } else {
-    prune_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint4*>(W), nvec, K / 8, nullptr,
-                                             mask_in, mask_out, n_keep);
+    return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K,
+                                                n_keep, nullptr, nullptr, s);
   }
-  return launch_status();
+  return launch_stream<true, false, kValsNone>(W, mask_in, mask_out, nullptr, nullptr, N, K,
+                                               n_keep, nullptr, nullptr, s);
 }
 
 sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const void* Xc,
@@ -581,10 +752,8 @@ sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const 
   SP24_TRY(noalloc_norms(&norms));
   cudaStream_t s = as_stream(stream);
   SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
-  const int64_t nvec = N * (K / 8);
-  prune_kernel<true><<<grid_for((nvec + 3) / 4, 256), 256, 0, s>>>(
-      static_cast<const uint4*>(W), nvec, K / 8, norms, mask_in, mask_out, n_keep);
-  return launch_status();
+  return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K, n_keep,
+                                              nullptr, nullptr, s);
 }
 
 sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K,
@@ -669,10 +838,10 @@ sp24_status sp24_compress(const void* W, const uint8_t* mask, int64_t N, int64_t
   SP24_TRY(check_device());
   cudaStream_t s = as_stream(stream);
   if (dtype == SP24_BF16)
-    return launch_compress<SP24_BF16, false, false>(W, mask, nullptr, nullptr, nullptr, nullptr, N,
-                                                     K, vals, meta, s);
-  return launch_compress<SP24_INT8, false, false>(W, mask, nullptr, nullptr, nullptr, s_w, N, K,
+    return launch_stream<false, false, kValsBF16>(W, mask, nullptr, nullptr, nullptr, N, K, 2,
                                                   vals, meta, s);
+  return launch_stream<false, false, kValsINT8>(W, mask, nullptr, nullptr, s_w, N, K, 2, vals,
+                                                meta, s);
 }
 
 sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
@@ -695,15 +864,15 @@ sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
   cudaStream_t s = as_stream(stream);
   const bool wanda = mode == SP24_WANDA;
   if (dtype == SP24_BF16) {
-    return wanda ? launch_compress<SP24_BF16, true, true>(W, nullptr, mask_in, mask_out, norms,
-                                                           nullptr, N, K, vals, meta, s)
-                 : launch_compress<SP24_BF16, true, false>(W, nullptr, mask_in, mask_out,
-                                                            nullptr, nullptr, N, K, vals, meta, s);
+    return wanda ? launch_stream<true, true, kValsBF16>(W, mask_in, mask_out, norms, nullptr, N, K,
+                                                        2, vals, meta, s)
+                 : launch_stream<true, false, kValsBF16>(W, mask_in, mask_out, nullptr, nullptr, N,
+                                                         K, 2, vals, meta, s);
   }
-  return wanda ? launch_compress<SP24_INT8, true, true>(W, nullptr, mask_in, mask_out, norms, s_w,
-                                                         N, K, vals, meta, s)
-               : launch_compress<SP24_INT8, true, false>(W, nullptr, mask_in, mask_out, nullptr,
-                                                          s_w, N, K, vals, meta, s);
+  return wanda ? launch_stream<true, true, kValsINT8>(W, mask_in, mask_out, norms, s_w, N, K, 2,
+                                                      vals, meta, s)
+               : launch_stream<true, false, kValsINT8>(W, mask_in, mask_out, nullptr, s_w, N, K,
+                                                       2, vals, meta, s);
 }
 
 }  // extern "C"
