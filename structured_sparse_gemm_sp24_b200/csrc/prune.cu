@@ -410,25 +410,56 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 }
 
 // --------------------------------------------------------- a5 weight scale
-// One CTA per row.  Keys = |w| bit patterns (15 bits) of the kept positions;
-// the r-th smallest key is found with two histogram passes (high 8 bits, then
-// low 7 bits within the selected bucket).
+// One warp per row (8 rows per 256-thread block).  Keys = |w| bit patterns (15
+// bits) of the kept positions.  One pass gives the kept count c and the
+// largest key; when the nearest rank r = ceil(coverage * c) equals c that is
+// the answer.  Otherwise the r-th smallest key is found exactly with two
+// histogram passes in the warp's shared-memory histogram (high 8 bits, then
+// low 7 bits inside the selected bucket) and warp-parallel prefix scans.
+
+// First bin b (of nb, lanes hold nb/32 consecutive bins each) whose inclusive
+// prefix count reaches `rank`; returns b and the count below it.
+__device__ __forceinline__ uint32_t warp_find_bin(const uint32_t* h, uint32_t nb, uint32_t rank,
+                                                  uint32_t& below) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t per = nb / 32u;
+  uint32_t local = 0;
+  for (uint32_t i = 0; i < per; ++i) local += h[lane * per + i];
+  uint32_t incl = local;   // inclusive warp scan of the lane totals
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= static_cast<uint32_t>(o)) incl += t;
+  }
+  const uint32_t excl = incl - local;
+  const uint32_t hit = __ballot_sync(0xFFFFFFFFu, incl >= rank && excl < rank);
+  const uint32_t src = __ffs(hit) - 1u;
+  uint32_t b = 0, acc = __shfl_sync(0xFFFFFFFFu, excl, src);
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t cnt = h[src * per + i];
+    if (acc + cnt >= rank) { b = src * per + i; break; }
+    acc += cnt;
+  }
+  below = acc;
+  return b;
+}
+
 __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict__ w,
-                                                     const uint8_t* __restrict__ mask,
+                                                     const uint8_t* __restrict__ mask, int64_t n,
                                                      int64_t k, double coverage,
                                                      float* __restrict__ s_w) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t s_count, s_bucket, s_rank;
-  const int64_t row = blockIdx.x;
+  __shared__ uint32_t hist[8][256];
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t wid = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + wid;
+  if (row >= n) return;                                  // whole warp leaves together
   const uint16_t* wr = w + row * k;
   const uint8_t* mr = mask + row * (k / 8);
   const int64_t kvec = k / 8;
+  uint32_t* h = hist[wid];
 
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-  if (threadIdx.x == 0) s_count = 0;
-  __syncthreads();
-  uint32_t cnt = 0;
-  for (int64_t v = threadIdx.x; v < kvec; v += blockDim.x) {
+  uint32_t cnt = 0, kmax = 0;
+  for (int64_t v = lane; v < kvec; v += 32) {
     const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
     const uint32_t keep = mr[v];
     const uint32_t words[4] = {q.x, q.y, q.z, q.w};
@@ -436,59 +467,62 @@ __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict_
     for (int i = 0; i < 8; ++i) {
       if ((keep >> i) & 1u) {
         const uint32_t key = mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]);
-        atomicAdd(&hist[key >> 7], 1u);
+        kmax = max(kmax, key);
         ++cnt;
       }
     }
   }
-  atomicAdd(&s_count, cnt);
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const uint32_t c = s_count;
-    uint32_t r = c == 0 ? 0u : static_cast<uint32_t>(ceil(coverage * static_cast<double>(c)));
-    if (r < 1) r = 1;
-    if (r > c) r = c;
-    uint32_t below = 0, b = 0;
-    for (b = 0; b < 256; ++b) {
-      if (below + hist[b] >= r) break;
-      below += hist[b];
-    }
-    s_bucket = b;
-    s_rank = r - below;  // rank within the bucket, 1-based
-  }
-  __syncthreads();
-  const uint32_t c = s_count;
-  const uint32_t bucket = s_bucket;
-  for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  if (c > 0) {
-    for (int64_t v = threadIdx.x; v < kvec; v += blockDim.x) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
-      const uint32_t keep = mr[v];
-      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if ((keep >> i) & 1u) {
-          const uint32_t key = mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]);
-          if ((key >> 7) == bucket) atomicAdd(&hist[key & 0x7Fu], 1u);
+  for (int o = 16; o > 0; o >>= 1) {
+    cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, o);
+    kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+  }
+  uint32_t key = 0;
+  if (cnt > 0) {
+    double rd = ceil(coverage * static_cast<double>(cnt));
+    uint32_t r = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
+    if (r > cnt) r = cnt;
+    if (r == cnt) {
+      key = kmax;
+    } else {
+      for (uint32_t i = lane; i < 256; i += 32) h[i] = 0;
+      __syncwarp();
+      for (int64_t v = lane; v < kvec; v += 32) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
+        const uint32_t keep = mr[v];
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if ((keep >> i) & 1u)
+            atomicAdd(&h[mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]) >> 7], 1u);
+      }
+      __syncwarp();
+      uint32_t below = 0;
+      const uint32_t bucket = warp_find_bin(h, 256, r, below);
+      const uint32_t r2 = r - below;
+      __syncwarp();
+      for (uint32_t i = lane; i < 256; i += 32) h[i] = 0;
+      __syncwarp();
+      for (int64_t v = lane; v < kvec; v += 32) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
+        const uint32_t keep = mr[v];
+        const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if ((keep >> i) & 1u) {
+            const uint32_t kk = mag_key((i & 1) ? (words[i / 2] >> 16) : words[i / 2]);
+            if ((kk >> 7) == bucket) atomicAdd(&h[kk & 0x7Fu], 1u);
+          }
         }
       }
+      __syncwarp();
+      uint32_t below2 = 0;
+      key = (bucket << 7) | warp_find_bin(h, 128, r2, below2);
     }
   }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float s = 1.0f;
-    if (c > 0) {
-      uint32_t below = 0, b = 0;
-      for (b = 0; b < 128; ++b) {
-        if (below + hist[b] >= s_rank) break;
-        below += hist[b];
-      }
-      const uint32_t key = (bucket << 7) | b;
-      const float t = __uint_as_float(key << 16);
-      if (t != 0.0f) s = __fdiv_rn(t, 127.0f);
-    }
-    s_w[row] = s;
+  if (lane == 0) {
+    const float t = __uint_as_float(key << 16);
+    s_w[row] = (cnt == 0 || t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
   }
 }
 
@@ -764,8 +798,8 @@ sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K
   if (K % 8 != 0 || !aligned16(W) || !aligned16(mask) || !aligned16(s_w)) return SP24_ERR_ALIGN;
   if (N > 0x7FFFFFFF) return SP24_ERR_ARG;
   SP24_TRY(check_device());
-  wscale_kernel<<<static_cast<unsigned>(N), 256, 0, as_stream(stream)>>>(
-      static_cast<const uint16_t*>(W), mask, K, coverage, s_w);
+  wscale_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, as_stream(stream)>>>(
+      static_cast<const uint16_t*>(W), mask, N, K, coverage, s_w);
   return launch_status();
 }
 
