@@ -18,7 +18,7 @@
 //  * tensor-memory full: multicast commit to both epilogues; tensor-memory
 //    empty: the even CTA's barrier collects one arrival per epilogue warp of
 //    both CTAs.
-// Warps: 0 = TMA producer (both CTAs), 1 = MMA issuer (even CTA), 2..5 =
+// Warps: 0 = TMA producer (both CTAs), 1 = MMA issuer (even CTA), 2..9 =
 // epilogue (both CTAs; warp 2 also owns the tensor-memory allocation).
 #pragma once
 
@@ -43,12 +43,10 @@ struct PairCfg {
                                    : kTmemNeeded <= 64 ? 64
                                    : kTmemNeeded <= 128 ? 128
                                    : kTmemNeeded <= 256 ? 256 : 512;
-  static constexpr int kOutBytes = OUTK == SP24_OUT_INT32 ? 4 : (OUTK == SP24_OUT_INT8 ? 1 : 2);
-  static constexpr int kChunk = 32;
-  static constexpr int kChBox = kOutBytes == 4 ? 64 : 128;
-  static constexpr int kStagingBytes = kChunk * 128 * kOutBytes;
+  static constexpr int kOutBytes = EpiOut<OUTK>::kBytes;
+  static constexpr int kStagingBytes = EpiOut<OUTK>::kStagingBytes;  // all epilogue warps
   static constexpr int kRingBytes = STAGES * kStageStride;
-  static constexpr int kSmemBytes = kRingBytes + 2 * kStagingBytes + 1024 + 256;
+  static constexpr int kSmemBytes = kRingBytes + kStagingBytes + 1024 + 256;
   static_assert(kTmemNeeded <= 512, "tensor memory overflow");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
   static_assert(kSmemBytes <= 232448, "shared memory");
@@ -63,7 +61,7 @@ __device__ __forceinline__ uint32_t make_idesc_pair(uint32_t id2) {
 }
 
 template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + kEpiThreads, 1)
 gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
              const PersistArgs args) {
@@ -72,7 +70,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* staging = smem + C::kRingBytes;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + 2 * C::kStagingBytes);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + C::kStagingBytes);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;
   uint64_t* tempty_bar = tfull_bar + C::kAcc;
@@ -94,7 +92,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
     for (int a = 0; a < C::kAcc; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 8);   // 4 epilogue warps x 2 CTAs
+      mbar_init(&tempty_bar[a], 2 * kEpiWarps);   // epilogue warps of both CTAs
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -188,75 +186,38 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
     }
   } else {
     // --------------------------------------------------------- epilogue
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    const int tid_e = threadIdx.x - 64;
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    const int ew = warp - 2;                 // 0..7
+    const int grp = ew >> 2;                 // which chunks of a tile (even / odd)
+    const int quad = warp & 3;               // tensor-memory lane quadrant of this warp
     const float sx = (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32) ? *args.s_x : 1.0f;
-    const float sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
-    const int ybox = args.y_box;
-    const int sidx = (row / ybox) * (C::kChunk * ybox) + (row % ybox);
-    uint32_t j = 0, chunk_ctr = 0;
+    EpiWarp e;
+    e.m = args.m;
+    e.n = args.n;
+    e.cbox = args.y_box;
+    e.vec = OUTK == SP24_OUT_BF16 && args.y_box == kEpiBox;
+    e.stg = staging + ew * EpiOut<OUTK>::kWarpBytes;
+    e.sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
+    uint32_t j = 0;
     for (int tile = pair; tile < ntiles; tile += npairs, ++j) {
       int prt, tt;
       tile_coords(tile, args, prt, tt);
       const int rt128 = prt * 2 + static_cast<int>(rank);
       const uint32_t acc = j % C::kAcc;
       bool ok = true;
-      if (tid_e == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
-      if (!named_barrier_and(1, 128, ok)) { *abort_flag = 1; break; }
+      if (lane == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const int64_t n_idx = static_cast<int64_t>(rt128) * 128 + row;
-      const bool row_valid = n_idx < args.n;
-      float cscale = 0.0f;
-      if constexpr (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32)
-        cscale = row_valid ? __fmul_rn(sx, __ldg(args.s_w + n_idx)) : 0.0f;
-      const int64_t tok0 = static_cast<int64_t>(tt) * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN / C::kChunk; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + acc * BN + c * C::kChunk, r);
-        tmem_ld_wait();
-        if (c == BN / C::kChunk - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(map_peer(smem_u32(&tempty_bar[acc]), 0));
-        }
-        if (tok0 + c * C::kChunk >= args.m) continue;
-        uint8_t* stg = staging + (chunk_ctr & 1u) * C::kStagingBytes;
-        if (tid_e == 0) bulk_wait_read<1>();
-        named_barrier(1, 128);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          if (!row_valid) break;
-          const int e = sidx + t * ybox;
-          if constexpr (kDtype == SP24_BF16) {
-            reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(__uint_as_float(r[t]));
-          } else if constexpr (OUTK == SP24_OUT_INT32) {
-            reinterpret_cast<uint32_t*>(stg)[e] = r[t];
-          } else {
-            const float f = __fmul_rn(__int2float_rn(static_cast<int32_t>(r[t])), cscale);
-            if constexpr (OUTK == SP24_OUT_BF16) {
-              reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(f);
-            } else {
-              int qv = __float2int_rn(__fdiv_rn(f, sy));
-              qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
-              reinterpret_cast<int8_t*>(stg)[e] = static_cast<int8_t>(qv);
-            }
-          }
-        }
-        fence_async_shared();
-        named_barrier(1, 128);
-        if (tid_e == 0) {
-          for (int bx = 0; bx * ybox < 128 && rt128 * 128 + bx * ybox < args.n; ++bx)
-            tma_store_2d(&tmap_y, stg + bx * (C::kChunk * ybox * C::kOutBytes),
-                         rt128 * 128 + bx * ybox, static_cast<int32_t>(tok0 + c * C::kChunk));
-          bulk_commit();
-        }
-        ++chunk_ctr;
-      }
+      e.c0 = rt128 * 128 + quad * 32;
+      epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
+      e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      e.tok0 = static_cast<int64_t>(tt) * BN;
+      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, grp, lane, [&] {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(map_peer(smem_u32(&tempty_bar[acc]), 0));
+      });
     }
-    if (tid_e == 0) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
   }
 
   __syncwarp();

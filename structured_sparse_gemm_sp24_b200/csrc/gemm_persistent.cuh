@@ -8,11 +8,9 @@
 //    tiles of a wave stay in L2 (each weight byte is fetched from HBM once);
 //  * two tensor-memory accumulators: the MMA warp fills one tile while the
 //    epilogue warps drain the other;
-//  * the epilogue drains 32 columns (tokens) at a time: tcgen05.ld -> cast /
-//    dequantise in registers -> shared-memory staging [32 tokens][128
-//    channels] -> TMA tensor store (clipped at the M / N edges), with two
-//    staging buffers so the store of one chunk overlaps the next.
-// Warps: 0 = TMA producer, 1 = MMA issuer, 2..5 = epilogue (warp 2 also owns
+//  * eight epilogue warps drain 32 tokens x 32 channels at a time, each with
+//    its own staging box and TMA store (the shared epilogue code).
+// Warps: 0 = TMA producer, 1 = MMA issuer, 2..9 = epilogue (warp 2 also owns
 // the tensor-memory allocation).
 #pragma once
 
@@ -36,15 +34,10 @@ struct PersistCfg {
                                    : kTmemNeeded <= 64 ? 64
                                    : kTmemNeeded <= 128 ? 128
                                    : kTmemNeeded <= 256 ? 256 : 512;
-  static constexpr int kOutBytes = OUTK == SP24_OUT_INT32 ? 4 : (OUTK == SP24_OUT_INT8 ? 1 : 2);
-  static constexpr int kChunk = 32;                              // tokens per epilogue chunk
-  // store box: [32 tokens][y_box channels], y_box = min(kChBox, N) (the
-  // tensor-map encoder rejects a box wider than the tensor), at most 256
-  // bytes per row; a staging buffer holds the boxes of one chunk back to back
-  static constexpr int kChBox = kOutBytes == 4 ? 64 : 128;
-  static constexpr int kStagingBytes = kChunk * 128 * kOutBytes;  // one staging buffer
+  static constexpr int kOutBytes = EpiOut<OUTK>::kBytes;
+  static constexpr int kStagingBytes = EpiOut<OUTK>::kStagingBytes;  // all epilogue warps
   static constexpr int kRingBytes = STAGES * kStageStride;
-  static constexpr int kSmemBytes = kRingBytes + 2 * kStagingBytes + 1024 + 256;
+  static constexpr int kSmemBytes = kRingBytes + kStagingBytes + 1024 + 256;
   static_assert(kTmemNeeded <= 512, "tensor memory overflow");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
   static_assert(kSmemBytes <= 232448, "shared memory");
@@ -60,7 +53,7 @@ struct PersistArgs {
   int row_tiles;     // ceil(N / 128)
   int tok_tiles;     // ceil(M / BN)
   int group_rows;    // raster group height (row tiles)
-  int y_box;         // channels per TMA store box: min(kChBox, N), a multiple of 8
+  int y_box;         // channels per epilogue store box: min(32, N)
 };
 
 // Linear tile index -> (row tile, token tile) in the grouped order.
@@ -75,7 +68,7 @@ __device__ __forceinline__ void tile_coords(int t, const PersistArgs& a, int& rt
 }
 
 template <int kDtype, int BN, int STAGES, int OUTK>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + kEpiThreads, 1)
 gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_y, const PersistArgs args) {
@@ -84,7 +77,7 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* staging = smem + C::kRingBytes;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + 2 * C::kStagingBytes);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(staging + C::kStagingBytes);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;
   uint64_t* tempty_bar = tfull_bar + C::kAcc;
@@ -102,7 +95,7 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
     }
     for (int a = 0; a < C::kAcc; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 4);   // one arrival per epilogue warp
+      mbar_init(&tempty_bar[a], kEpiWarps);   // one arrival per epilogue warp
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -197,78 +190,37 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
     }
   } else {
     // --------------------------------------------------------- epilogue
+    const int ew = warp - 2;                 // 0..7
+    const int grp = ew >> 2;                 // which chunks of a tile (even / odd)
     const int quad = warp & 3;               // tensor-memory lane quadrant of this warp
-    const int row = quad * 32 + lane;        // output channel within the tile
-    const int tid_e = threadIdx.x - 64;      // 0..127
-    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
     const float sx = (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32) ? *args.s_x : 1.0f;
-    const float sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
-    // staging element of (token 0, this channel): box row / ybox, column row % ybox
-    const int ybox = args.y_box;
-    const int sidx = (row / ybox) * (C::kChunk * ybox) + (row % ybox);
-    uint32_t j = 0, chunk_ctr = 0;
+    EpiWarp e;
+    e.m = args.m;
+    e.n = args.n;
+    e.cbox = args.y_box;
+    e.vec = OUTK == SP24_OUT_BF16 && args.y_box == kEpiBox;
+    e.stg = staging + ew * EpiOut<OUTK>::kWarpBytes;
+    e.sy = (kDtype == SP24_INT8 && OUTK == SP24_OUT_INT8) ? *args.s_y : 1.0f;
+    uint32_t j = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++j) {
       int rt, tt;
       tile_coords(tile, args, rt, tt);
       const uint32_t acc = j % C::kAcc;
       bool ok = true;
-      if (tid_e == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
-      if (!named_barrier_and(1, 128, ok)) { *abort_flag = 1; break; }
+      if (lane == 0) ok = !*abort_flag && mbar_wait(&tfull_bar[acc], (j / C::kAcc) & 1u);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) { *abort_flag = 1; break; }
       tc_fence_after();
-      const int64_t n_idx = static_cast<int64_t>(rt) * 128 + row;
-      const bool row_valid = n_idx < args.n;
-      float cscale = 0.0f;
-      if constexpr (kDtype == SP24_INT8 && OUTK != SP24_OUT_INT32)
-        cscale = n_idx < args.n ? __fmul_rn(sx, __ldg(args.s_w + n_idx)) : 0.0f;
-      const int64_t tok0 = static_cast<int64_t>(tt) * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN / C::kChunk; ++c) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + acc * BN + c * C::kChunk, r);
-        tmem_ld_wait();
-        if (c == BN / C::kChunk - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty_bar[acc]);   // accumulator drained
-        }
-        if (tok0 + c * C::kChunk >= args.m) continue;       // chunk entirely past M
-        uint8_t* stg = staging + (chunk_ctr & 1u) * C::kStagingBytes;
-        if (tid_e == 0) bulk_wait_read<1>();                 // buffer's previous store done
-        named_barrier(1, 128);
-        // channels at or past N are never stored (and, when N < 128, would
-        // index past the staging buffer): skip them
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          if (!row_valid) break;
-          const int e = sidx + t * ybox;
-          if constexpr (kDtype == SP24_BF16) {
-            const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(r[t]));
-            reinterpret_cast<__nv_bfloat16*>(stg)[e] = h;
-          } else if constexpr (OUTK == SP24_OUT_INT32) {
-            reinterpret_cast<uint32_t*>(stg)[e] = r[t];
-          } else {
-            const float f = __fmul_rn(__int2float_rn(static_cast<int32_t>(r[t])), cscale);
-            if constexpr (OUTK == SP24_OUT_BF16) {
-              reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(f);
-            } else {
-              int qv = __float2int_rn(__fdiv_rn(f, sy));
-              qv = qv > 127 ? 127 : (qv < -127 ? -127 : qv);
-              reinterpret_cast<int8_t*>(stg)[e] = static_cast<int8_t>(qv);
-            }
-          }
-        }
-        fence_async_shared();
-        named_barrier(1, 128);
-        if (tid_e == 0) {
-          for (int bx = 0; bx * ybox < 128 && rt * 128 + bx * ybox < args.n; ++bx)
-            tma_store_2d(&tmap_y, stg + bx * (C::kChunk * ybox * C::kOutBytes),
-                         rt * 128 + bx * ybox, static_cast<int32_t>(tok0 + c * C::kChunk));
-          bulk_commit();
-        }
-        ++chunk_ctr;
-      }
+      e.c0 = rt * 128 + quad * 32;
+      epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
+      e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
+      e.tok0 = static_cast<int64_t>(tt) * BN;
+      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, grp, lane, [&] {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty_bar[acc]);   // accumulator drained
+      });
     }
-    if (tid_e == 0) bulk_wait<0>();
+    if (lane == 0) bulk_wait<0>();
   }
 
   __syncwarp();

@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -316,6 +317,7 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
 }  // namespace sp24
 
+#include "gemm_epilogue.cuh"
 #include "gemm_persistent.cuh"
 #include "gemm_pair.cuh"
 
@@ -378,11 +380,11 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
   const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                   : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int y_box = static_cast<int>(g.n < C::kChBox ? g.n : C::kChBox);
+  const int y_box = epi_box(g.n);
   CUtensorMap my;
   SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
-                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), C::kChunk,
-                    CU_TENSOR_MAP_SWIZZLE_NONE));
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk,
+                    epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE));
   PersistArgs a;
   a.meta = g.meta;
   a.s_x = g.s_x;
@@ -403,7 +405,7 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
   const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
   if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(ntiles < sm_count() ? ntiles : sm_count());
-  kern<<<grid, 192, C::kSmemBytes, s>>>(ma, mb, my, a);
+  kern<<<grid, 64 + kEpiThreads, C::kSmemBytes, s>>>(ma, mb, my, a);
   return launch_status();
 }
 
@@ -440,11 +442,11 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                   : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  const int y_box = static_cast<int>(g.n < C::kChBox ? g.n : C::kChBox);
+  const int y_box = epi_box(g.n);
   CUtensorMap my;
   SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
-                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), C::kChunk,
-                    CU_TENSOR_MAP_SWIZZLE_NONE));
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk,
+                    epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE));
   PersistArgs a;
   a.meta = g.meta;
   a.s_x = g.s_x;
@@ -467,7 +469,7 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   const int pairs = static_cast<int>(ntiles < max_pairs ? ntiles : max_pairs);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(64 + kEpiThreads, 1, 1);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -482,27 +484,67 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   return launch_status();
 }
 
-// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair128 |
-// single (tuning override; default chooses by problem size).
+// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair224 |
+// pair192 | pair128 | single (tuning override; default chooses by problem size).
 int impl_choice() {
   const char* e = std::getenv("SP24_GEMM_IMPL");
   if (!e) return 0;
   if (std::strcmp(e, "pair256") == 0) return 1;
   if (std::strcmp(e, "pair128") == 0) return 2;
   if (std::strcmp(e, "single") == 0) return 3;
+  if (std::strcmp(e, "pair224") == 0) return 4;
+  if (std::strcmp(e, "pair192") == 0) return 5;
   return 0;
 }
 
-// Tile plan: BN from the token count, split-K from how many tiles exist.
+// CTA-pair kernel for every output kind; ST = ring stages (ST32 with int32
+// output, whose staging is twice the size).
+template <int kDtype, int BN, int ST, int ST32, int ACC>
+sp24_status launch_pair_out(const CUtensorMap& ma, const GemmArgs& a, const void* x,
+                            cudaStream_t s) {
+  if constexpr (kDtype == SP24_BF16) {
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, s);
+  } else {
+    if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, BN, ST32, SP24_OUT_INT32, ACC>(ma, a, x, s);
+    if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, BN, ST, SP24_OUT_INT8, ACC>(ma, a, x, s);
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, s);
+  }
+}
+
+// Estimated run time (us, B200 under load) of a persistent variant: waves of
+// output tiles over the SMs (pairs) x per-tile time, i.e. k-blocks x the
+// measured cost of one k-block plus the part of the epilogue the variant
+// cannot overlap with the next tile.  Used only to rank the variants.
+double est_time(int impl, int64_t m, int64_t n, int kblocks, int sms) {
+  const auto waves = [](int64_t tiles, int64_t units) {
+    return static_cast<double>((tiles + units - 1) / units);
+  };
+  const double kb = kblocks;
+  switch (impl) {
+    case 1:   // 256 x 256 pair tile, one accumulator: whole epilogue exposed
+      return waves(((n + 255) / 256) * ((m + 255) / 256), sms / 2) * (0.50 * kb + 2.5);
+    case 4:   // 256 x 224 pair tile, two accumulators: only the last drain exposed
+      return waves(((n + 255) / 256) * ((m + 223) / 224), sms / 2) * std::max(0.50 * kb, 1.4) + 2.0;
+    default:  // 128 x 128 single-SM tile, two accumulators
+      return waves(((n + 127) / 128) * ((m + 127) / 128), sms) * std::max(0.48 * kb, 1.6);
+  }
+}
+
+// Tile plan.  At least 128 tokens and enough 128 x 128 tiles for half the SMs:
+// a persistent kernel, the variant with the lowest estimated time (or the
+// SP24_GEMM_IMPL override).  Otherwise (few tokens or few tiles): the split-K
+// kernel, BN from the token count and K split until the CTAs cover the SMs.
 template <int kDtype>
 sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s) {
   const int sms = sm_count();
   const int64_t row_tiles = (a.n + 127) / 128;
+  const bool persistent = a.m >= 128 && row_tiles * ((a.m + 127) / 128) >= sms / 2;
   int bn = a.m <= 16 ? 16 : a.m <= 32 ? 32 : a.m <= 64 ? 64 : 128;
   const int64_t tok_tiles = (a.m + bn - 1) / bn;
   const int64_t base = row_tiles * tok_tiles;
   int split = 1;
-  while (split < 8 && base * split < 2 * sms && a.kblocks >= 2 * split) split *= 2;
+  if (!persistent)
+    while (split < 8 && base * split < 2 * sms && a.kblocks >= 2 * split) split *= 2;
   a.kb_per_split = (a.kblocks + split - 1) / split;
 
   const int el = kDtype == SP24_BF16 ? 2 : 1;
@@ -515,21 +557,22 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
   SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.m),
                     box_cols, static_cast<uint32_t>(bn)));
 
-  if (split == 1 && bn == 128) {
+  if (persistent) {
     int impl = impl_choice();
-    // pairs pay off once each tile has a long K loop (measured on B200: the
-    // 256 x 256 pair tile wins for K >= 1024 with M, N >= 512; short-K or
-    // narrow-N problems such as K = 768 or N = 64 are faster on single SMs)
-    if (impl == 0) impl = (a.kblocks >= 8 && a.m >= 512 && a.n >= 512) ? 1 : 3;
-    if (impl == 1) {
-      if constexpr (kDtype == SP24_BF16) {
-        return launch_pair<kDtype, 256, 4, SP24_OUT_BF16, 1>(ma, a, x, s);
-      } else {
-        if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, 256, 3, SP24_OUT_INT32, 1>(ma, a, x, s);
-        if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, 256, 4, SP24_OUT_INT8, 1>(ma, a, x, s);
-        return launch_pair<kDtype, 256, 4, SP24_OUT_BF16, 1>(ma, a, x, s);
+    if (impl == 0) {
+      // pair tiles need both dimensions to fill them
+      impl = 3;
+      if (a.m >= 256 && a.n >= 256) {
+        double best = est_time(3, a.m, a.n, a.kblocks, sms);
+        for (int c : {1, 4}) {
+          const double t = est_time(c, a.m, a.n, a.kblocks, sms);
+          if (t < best) { best = t; impl = c; }
+        }
       }
     }
+    if (impl == 1) return launch_pair_out<kDtype, 256, 4, 3, 1>(ma, a, x, s);
+    if (impl == 4) return launch_pair_out<kDtype, 224, 4, 4, 2>(ma, a, x, s);
+    if (impl == 5) return launch_pair_out<kDtype, 192, 4, 4, 2>(ma, a, x, s);
     if (impl == 2) {
       if constexpr (kDtype == SP24_BF16) {
         return launch_pair<kDtype, 128, 6, SP24_OUT_BF16, 2>(ma, a, x, s);

@@ -277,6 +277,36 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// 16 lanes x 32 columns starting at (lane, column) `taddr` into r[16*H ..
+// 16*H + 15]: register 4b + i of thread t holds lane t/4 + 8*(i>>1), column
+// 8b + 2*(t%4) + (i&1) (the accumulator fragment layout of mma / stmatrix).
+template <int H>
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[16 * H + 0]), "=r"(r[16 * H + 1]), "=r"(r[16 * H + 2]), "=r"(r[16 * H + 3]),
+        "=r"(r[16 * H + 4]), "=r"(r[16 * H + 5]), "=r"(r[16 * H + 6]), "=r"(r[16 * H + 7]),
+        "=r"(r[16 * H + 8]), "=r"(r[16 * H + 9]), "=r"(r[16 * H + 10]), "=r"(r[16 * H + 11]),
+        "=r"(r[16 * H + 12]), "=r"(r[16 * H + 13]), "=r"(r[16 * H + 14]), "=r"(r[16 * H + 15])
+      : "r"(taddr));
+}
+
+// Four 8x8 b16 matrices, each stored transposed: fragment element (row c, col
+// r) -- held by thread 4c + r/2 in half r&1 of register `a<m>` -- lands at
+// position c of shared row r of matrix m, whose 16-byte address thread 8m + r
+// supplies.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a0, uint32_t a1,
+                                                  uint32_t a2, uint32_t a3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
+               ::"r"(saddr), "r"(a0), "r"(a1), "r"(a2), "r"(a3) : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 
 // ------------------------------------------------- CTA-pair (cta_group::2)
 // The two CTAs of a cluster of 2 act as one MMA unit: the even CTA issues
@@ -347,9 +377,12 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint64_t* bar, uint16_t cta_ma
 }
 
 // Arrive on an mbarrier in another CTA of the cluster (cluster address).
+// Arrive on an mbarrier of a CTA of this cluster (default .release.cta
+// semantics).  Used where the arrival hands over tensor memory whose reads
+// are already complete (tcgen05.wait::ld + tcgen05 fence), so no
+// cluster-scope ordering of this thread's memory operations is needed.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];"
-               ::"r"(bar_cluster) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
 
 // ------------------------------------------------------------------ cluster

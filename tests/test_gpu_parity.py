@@ -424,7 +424,7 @@ def gemm_impl(request, monkeypatch):
     return request.param
 
 
-@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair256"], indirect=True)
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair256"], indirect=True)
 @pytest.mark.parametrize("mnk", IMPL_SHAPES)
 def test_gemm_bf16_impls(gemm_impl, mnk):
     m, n, k = mnk
@@ -435,7 +435,7 @@ def test_gemm_bf16_impls(gemm_impl, mnk):
     ok_status()
 
 
-@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair256"], indirect=True)
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair256"], indirect=True)
 @pytest.mark.parametrize("out_kind", [B.SP24_OUT_INT32, B.SP24_OUT_BF16, B.SP24_OUT_INT8])
 @pytest.mark.parametrize("mnk", [(2500, 2064, 416), (130, 528, 96 + 32), (3000, 1808, 1280)])
 def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
