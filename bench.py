@@ -477,7 +477,9 @@ def main(argv=None):
     roof["traffic"] = None
     roof["peak_source"] = peaks["source"] + (" (2x dense bf16 burst)" if not wl.int8 else
                                              " (4x dense bf16 burst)")
-    roof["kernel"] = "gemm_sp_kernel"
+    plan = B.sp24_gemm_plan(wl.M, wl.N, wl.K, B.SP24_INT8 if wl.int8 else B.SP24_BF16)
+    roof["kernel"] = "sp24 gemm " + plan["kernel"]
+    roof["plan"] = plan
     c_gbs = runner.compress_bytes() / (comp_ms * 1e-3) / 1e9
 
     line = {

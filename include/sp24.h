@@ -203,6 +203,32 @@ sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
                       const float* s_w, int out_kind, const float* s_y, void* Y,
                       void* stream);
 
+/* The launch sp24_gemm makes for an M x N x K problem of `dtype` on the
+ * current device (the pages fix no kernel design; this reports the one this
+ * library chose, for profiling and tests).  Fills *plan; allocates nothing
+ * and launches nothing.  The SP24_GEMM_IMPL environment variable, if set
+ * (pair256, pair240, pair224, pair192, pair128, single), overrides the
+ * persistent-kernel choice exactly as it does for sp24_gemm.
+ *   kernel:        "splitk" (few tokens or tiles: K split across a cluster),
+ *                  "single" (persistent, one 128 x 128 tile per SM at a time),
+ *                  "pairNNN" (persistent, a CTA pair on two SMs computes
+ *                  256-channel x NNN-token tiles with tcgen05 cta_group::2).
+ *   tile_tokens, tile_channels: output tile (rows of Y x columns of Y).
+ *   split_k:       K slices per tile (1 unless "splitk").
+ *   ctas, cluster: CTAs launched and CTAs per cluster.
+ * Errors: SP24_ERR_ARG for a NULL plan, M < 1, N < 1, K < 16 or an unknown
+ * dtype; SP24_ERR_CUDA if the device cannot be queried. */
+typedef struct sp24_gemm_plan_t {
+  char kernel[16];
+  int32_t tile_tokens;
+  int32_t tile_channels;
+  int32_t split_k;
+  int32_t cluster;
+  int64_t ctas;
+} sp24_gemm_plan_t;
+
+sp24_status sp24_gemm_plan(int64_t M, int64_t N, int64_t K, int dtype, sp24_gemm_plan_t* plan);
+
 /* ------------------------------------------------- allocation-free variant */
 
 /* Largest K accepted by sp24_prune_wanda_noalloc. */

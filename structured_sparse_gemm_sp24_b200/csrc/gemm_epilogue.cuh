@@ -65,11 +65,11 @@ __device__ __forceinline__ float epi_value(uint32_t acc, float cscale) {
 // tokens 8b ..).  Thread `lane` addresses token row 8b + lane%8 of matrix
 // lane/8 for stmatrix; the box row is 64 bytes and its 16-byte chunk index is
 // XORed with bits 1-2 of the row (64-byte swizzle).
-template <int kDtype>
+template <int kDtype, int NB>
 __device__ __forceinline__ void stage_vec(const uint32_t (&r)[32], uint32_t stg, int lane,
                                           const float (&cs)[4]) {
 #pragma unroll
-  for (int b = 0; b < 4; ++b) {
+  for (int b = 0; b < NB; ++b) {
     uint32_t p[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -82,12 +82,12 @@ __device__ __forceinline__ void stage_vec(const uint32_t (&r)[32], uint32_t stg,
   }
 }
 
-// One-channel-per-thread path (thread `lane` owns channel c0 + lane).
-template <int kDtype, int OUTK>
+// One-channel-per-thread path (thread `lane` owns channel c0 + lane), NT tokens.
+template <int kDtype, int OUTK, int NT>
 __device__ __forceinline__ void stage_scalar(const uint32_t (&r)[32], uint8_t* stg, int lane,
                                              int cbox, float cscale, float sy) {
 #pragma unroll
-  for (int t = 0; t < 32; ++t) {
+  for (int t = 0; t < NT; ++t) {
     const int e = t * cbox + lane;
     if constexpr (kDtype == SP24_BF16) {
       reinterpret_cast<__nv_bfloat16*>(stg)[e] = __float2bfloat16_rn(__uint_as_float(r[t]));
@@ -106,48 +106,65 @@ __device__ __forceinline__ void stage_scalar(const uint32_t (&r)[32], uint8_t* s
   }
 }
 
-__device__ __forceinline__ void epi_load(const EpiWarp& e, int chunk, uint32_t (&r)[32]) {
+__device__ __forceinline__ void epi_load(const EpiWarp& e, int chunk, bool half,
+                                         uint32_t (&r)[32]) {
   const uint32_t ta = e.tmem + static_cast<uint32_t>(chunk * kEpiChunk);
   if (e.vec) {
-    tmem_ld_16x256b_x4<0>(ta, r);
-    tmem_ld_16x256b_x4<1>(ta + (16u << 16), r);
+    if (half) {
+      tmem_ld_16x256b_x2<0>(ta, r);
+      tmem_ld_16x256b_x2<1>(ta + (16u << 16), r);
+    } else {
+      tmem_ld_16x256b_x4<0>(ta, r);
+      tmem_ld_16x256b_x4<1>(ta + (16u << 16), r);
+    }
+  } else if (half) {
+    tmem_ld16_into(ta, r);
   } else {
     tmem_ld32(ta, r);
   }
 }
 
-// Drains this warp's chunks (grp, grp + 2, ...) of one tile.  `release` runs
-// once the warp's last tensor-memory load has completed (the accumulator may
-// then be reused); all lanes call it.
+// Drains this warp's chunks (grp, grp + 2, ...) of one tile.  With BN % 32 ==
+// 16 the tile's last chunk holds 16 tokens and is stored through `tmap_y16`
+// (16-token boxes), so no store reaches past the tile.  `release` runs once
+// the warp's last tensor-memory load has completed (the accumulator may then
+// be reused); all lanes call it.
 template <int kDtype, int OUTK, int BN, class Release>
 __device__ __forceinline__ void epilogue_tile(const EpiWarp& e, const CUtensorMap* tmap_y,
-                                              int grp, int lane, Release&& release) {
-  constexpr int kChunks = BN / kEpiChunk;
+                                              const CUtensorMap* tmap_y16, int grp, int lane,
+                                              Release&& release) {
+  static_assert(BN % 16 == 0, "tile width");
+  constexpr int kChunks = (BN + kEpiChunk - 1) / kEpiChunk;
+  constexpr bool kHalfTail = BN % kEpiChunk != 0;
   static_assert(kChunks >= 2, "each warp of a quadrant must own a chunk of every tile");
   constexpr int kMaxMine = (kChunks + 1) / 2;
   const int nmine = (kChunks - grp + 1) / 2;
   const bool live = e.c0 < e.n;   // some channel of this quadrant exists
   uint32_t r[2][32];
-  if (nmine > 0) epi_load(e, grp, r[0]);
+  if (nmine > 0) epi_load(e, grp, kHalfTail && grp == kChunks - 1, r[0]);
 #pragma unroll
   for (int i = 0; i < kMaxMine; ++i) {
     if (i < nmine) {
+      const int c = grp + 2 * i;
+      const bool half = kHalfTail && c == kChunks - 1;
       tmem_ld_wait();   // chunk i landed (and nothing else is outstanding)
-      if (i + 1 < nmine) epi_load(e, grp + 2 * (i + 1), r[(i + 1) & 1]);
+      if (i + 1 < nmine) epi_load(e, c + 2, kHalfTail && c + 2 == kChunks - 1, r[(i + 1) & 1]);
       else release();
-      const int64_t t0 = e.tok0 + (grp + 2 * i) * kEpiChunk;
+      const int64_t t0 = e.tok0 + c * kEpiChunk;
       if (live && t0 < e.m) {
         if (lane == 0) bulk_wait_read<0>();         // this warp's previous store read out
         __syncwarp();
         if (e.vec) {
-          stage_vec<kDtype>(r[i & 1], smem_u32(e.stg), lane, e.cs);
+          if (half) stage_vec<kDtype, 2>(r[i & 1], smem_u32(e.stg), lane, e.cs);
+          else stage_vec<kDtype, 4>(r[i & 1], smem_u32(e.stg), lane, e.cs);
         } else if (e.c0 + lane < e.n) {
-          stage_scalar<kDtype, OUTK>(r[i & 1], e.stg, lane, e.cbox, e.cs[0], e.sy);
+          if (half) stage_scalar<kDtype, OUTK, 16>(r[i & 1], e.stg, lane, e.cbox, e.cs[0], e.sy);
+          else stage_scalar<kDtype, OUTK, 32>(r[i & 1], e.stg, lane, e.cbox, e.cs[0], e.sy);
         }
         fence_async_shared();
         __syncwarp();
         if (lane == 0) {
-          tma_store_2d(tmap_y, e.stg, e.c0, static_cast<int32_t>(t0));
+          tma_store_2d(half ? tmap_y16 : tmap_y, e.stg, e.c0, static_cast<int32_t>(t0));
           bulk_commit();
         }
       }

@@ -48,7 +48,7 @@ struct PairCfg {
   static constexpr int kRingBytes = STAGES * kStageStride;
   static constexpr int kSmemBytes = kRingBytes + kStagingBytes + 1024 + 256;
   static_assert(kTmemNeeded <= 512, "tensor memory overflow");
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(BN % 16 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -64,7 +64,7 @@ template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
-             const PersistArgs args) {
+             const __grid_constant__ CUtensorMap tmap_y16, const PersistArgs args) {
   using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -211,7 +211,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
       e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       e.tok0 = static_cast<int64_t>(tt) * BN;
-      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, grp, lane, [&] {
+      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, &tmap_y16, grp, lane, [&] {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(map_peer(smem_u32(&tempty_bar[acc]), 0));

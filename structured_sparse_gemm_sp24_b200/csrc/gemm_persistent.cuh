@@ -39,7 +39,7 @@ struct PersistCfg {
   static constexpr int kRingBytes = STAGES * kStageStride;
   static constexpr int kSmemBytes = kRingBytes + kStagingBytes + 1024 + 256;
   static_assert(kTmemNeeded <= 512, "tensor memory overflow");
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
@@ -214,7 +214,7 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
       epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
       e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       e.tok0 = static_cast<int64_t>(tt) * BN;
-      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, grp, lane, [&] {
+      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, &tmap_y, grp, lane, [&] {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty_bar[acc]);   // accumulator drained

@@ -411,7 +411,7 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
 
 
 template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
-sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
+sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x, int pairs,
                         cudaStream_t s) {
   using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
   auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC>;
@@ -443,10 +443,18 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
                                   : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const int y_box = epi_box(g.n);
-  CUtensorMap my;
+  const CUtensorMapSwizzle yswz =
+      epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap my, my16;
   SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
-                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk,
-                    epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE));
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk, yswz));
+  // tiles of 16 (mod 32) tokens store their last chunk with 16-token boxes
+  if (BN % kEpiChunk != 0) {
+    SP24_TRY(make_map(&my16, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                      static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), 16, yswz));
+  } else {
+    my16 = my;
+  }
   PersistArgs a;
   a.meta = g.meta;
   a.s_x = g.s_x;
@@ -465,8 +473,7 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   a.y_box = y_box;
   const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
   if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
-  const int64_t max_pairs = sm_count() / 2;
-  const int pairs = static_cast<int>(ntiles < max_pairs ? ntiles : max_pairs);
+  if (pairs < 1 || pairs > ntiles) return SP24_ERR_ARG;   // the plan sizes the grid
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(64 + kEpiThreads, 1, 1);
@@ -479,74 +486,201 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, me, my, a);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, me, my, my16, a);
   if (le != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", le);
   return launch_status();
 }
 
-// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair224 |
-// pair192 | pair128 | single (tuning override; default chooses by problem size).
-int impl_choice() {
+// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair240 |
+// pair224 | pair192 | pair128 | single (tuning override; default chooses by
+// problem size).
+enum Impl : int { kSplitK = 0, kPair256 = 1, kPair128 = 2, kSingle = 3, kPair224 = 4,
+                  kPair192 = 5, kPair240 = 6 };
+
+int impl_override() {
   const char* e = std::getenv("SP24_GEMM_IMPL");
-  if (!e) return 0;
-  if (std::strcmp(e, "pair256") == 0) return 1;
-  if (std::strcmp(e, "pair128") == 0) return 2;
-  if (std::strcmp(e, "single") == 0) return 3;
-  if (std::strcmp(e, "pair224") == 0) return 4;
-  if (std::strcmp(e, "pair192") == 0) return 5;
-  return 0;
+  if (!e) return -1;
+  if (std::strcmp(e, "pair256") == 0) return kPair256;
+  if (std::strcmp(e, "pair128") == 0) return kPair128;
+  if (std::strcmp(e, "single") == 0) return kSingle;
+  if (std::strcmp(e, "pair224") == 0) return kPair224;
+  if (std::strcmp(e, "pair192") == 0) return kPair192;
+  if (std::strcmp(e, "pair240") == 0) return kPair240;
+  return -1;
+}
+
+const char* impl_name(int impl) {
+  switch (impl) {
+    case kPair256: return "pair256";
+    case kPair240: return "pair240";
+    case kPair224: return "pair224";
+    case kPair192: return "pair192";
+    case kPair128: return "pair128";
+    case kSingle: return "single";
+    default: return "splitk";
+  }
+}
+
+int pair_tokens(int impl) {
+  switch (impl) {
+    case kPair256: return 256;
+    case kPair240: return 240;
+    case kPair224: return 224;
+    case kPair192: return 192;
+    default: return 128;
+  }
+}
+
+// CTA pairs (clusters of 2) that can be resident at once.  A cluster lives in
+// one GPC, so a GPC with an odd number of SMs leaves one out and the count can
+// be below SMs / 2; the persistent pair kernels launch exactly this many pairs
+// so that no pair waits for another to finish.  Every pair variant holds one
+// CTA per SM, so one query (cached per device) serves them all.
+sp24_status pair_capacity(int* out) {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  if (cache[dev & 63] > 0) {
+    *out = cache[dev & 63];
+    return SP24_OK;
+  }
+  using C = PairCfg<SP24_BF16, 256, 4, SP24_OUT_BF16, 1>;
+  auto kern = gemm_sp_pair<SP24_BF16, 256, 4, SP24_OUT_BF16, 1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+  cfg.blockDim = dim3(64 + kEpiThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters", e);
+  if (n < 1) return SP24_ERR_UNSUPPORTED;
+  cache[dev & 63] = n;
+  *out = n;
+  return SP24_OK;
+}
+
+// Estimated run time (us, B200 under load) of a persistent variant: waves of
+// output tiles over the SMs (resident pairs) x per-tile time, i.e. k-blocks x
+// the measured cost of one k-block plus the part of the epilogue the variant
+// cannot overlap with the next tile.  Used only to rank the variants.
+double est_time(int impl, int64_t m, int64_t n, int kblocks, int sms, int pairs) {
+  const auto waves = [](int64_t tiles, int64_t units) {
+    return static_cast<double>((tiles + units - 1) / units);
+  };
+  const double kb = kblocks;
+  const int64_t prow = (n + 255) / 256;
+  switch (impl) {
+    case kPair256:   // one accumulator: the whole epilogue is exposed
+      return waves(prow * ((m + 255) / 256), pairs) * (0.50 * kb + 2.5);
+    case kPair240:   // two accumulators: only the last drain is exposed
+      return waves(prow * ((m + 239) / 240), pairs) * std::max(0.50 * kb, 1.5) + 2.0;
+    case kPair224:
+      return waves(prow * ((m + 223) / 224), pairs) * std::max(0.50 * kb, 1.4) + 2.0;
+    default:         // 128 x 128 single-SM tile, two accumulators
+      return waves(((n + 127) / 128) * ((m + 127) / 128), sms) * std::max(0.48 * kb, 1.6);
+  }
+}
+
+struct Plan {
+  int impl;            // Impl
+  int bn;              // split-K kernel: tokens per tile
+  int split;           // split-K kernel: K slices (= cluster size)
+  int64_t ctas;        // CTAs launched
+  int cluster;         // CTAs per cluster
+  int tile_tokens;     // tokens (rows of X and Y) per output tile
+  int tile_channels;   // output channels (rows of W) per output tile
+};
+
+// The launch plan.  At least 128 tokens and enough 128 x 128 tiles for half
+// the SMs: a persistent kernel, the variant with the lowest estimated time (or
+// the SP24_GEMM_IMPL override).  Otherwise (few tokens or few tiles): the
+// split-K kernel, BN from the token count and K split until the CTAs cover
+// the SMs.
+sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
+  const int sms = sm_count();
+  const int64_t row_tiles = (n + 127) / 128;
+  if (m >= 128 && row_tiles * ((m + 127) / 128) >= sms / 2) {
+    int pairs = 0;
+    SP24_TRY(pair_capacity(&pairs));
+    int impl = impl_override();
+    if (impl < 0) {
+      impl = kSingle;   // pair tiles need both dimensions to fill them
+      if (m >= 256 && n >= 256) {
+        double best = est_time(kSingle, m, n, kblocks, sms, pairs);
+        for (int c : {kPair256, kPair240, kPair224}) {
+          const double t = est_time(c, m, n, kblocks, sms, pairs);
+          if (t < best) {
+            best = t;
+            impl = c;
+          }
+        }
+      }
+    }
+    p->impl = impl;
+    p->bn = 128;
+    p->split = 1;
+    if (impl == kSingle) {
+      const int64_t tiles = row_tiles * ((m + 127) / 128);
+      p->ctas = tiles < sms ? tiles : sms;
+      p->cluster = 1;
+      p->tile_tokens = 128;
+      p->tile_channels = 128;
+    } else {
+      const int tok = pair_tokens(impl);
+      const int64_t tiles = ((n + 255) / 256) * ((m + tok - 1) / tok);
+      p->ctas = 2 * (tiles < pairs ? tiles : pairs);
+      p->cluster = 2;
+      p->tile_tokens = tok;
+      p->tile_channels = 256;
+    }
+    return SP24_OK;
+  }
+  const int bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
+  const int64_t base = row_tiles * ((m + bn - 1) / bn);
+  int split = 1;
+  while (split < 8 && base * split < 2 * sms && kblocks >= 2 * split) split *= 2;
+  p->impl = kSplitK;
+  p->bn = bn;
+  p->split = split;
+  p->ctas = base * split;
+  p->cluster = split;
+  p->tile_tokens = bn;
+  p->tile_channels = 128;
+  return SP24_OK;
 }
 
 // CTA-pair kernel for every output kind; ST = ring stages (ST32 with int32
 // output, whose staging is twice the size).
 template <int kDtype, int BN, int ST, int ST32, int ACC>
-sp24_status launch_pair_out(const CUtensorMap& ma, const GemmArgs& a, const void* x,
+sp24_status launch_pair_out(const CUtensorMap& ma, const GemmArgs& a, const void* x, int pairs,
                             cudaStream_t s) {
   if constexpr (kDtype == SP24_BF16) {
-    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, s);
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, pairs, s);
   } else {
-    if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, BN, ST32, SP24_OUT_INT32, ACC>(ma, a, x, s);
-    if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, BN, ST, SP24_OUT_INT8, ACC>(ma, a, x, s);
-    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, s);
+    if (a.out_kind == SP24_OUT_INT32)
+      return launch_pair<kDtype, BN, ST32, SP24_OUT_INT32, ACC>(ma, a, x, pairs, s);
+    if (a.out_kind == SP24_OUT_INT8)
+      return launch_pair<kDtype, BN, ST, SP24_OUT_INT8, ACC>(ma, a, x, pairs, s);
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, pairs, s);
   }
 }
 
-// Estimated run time (us, B200 under load) of a persistent variant: waves of
-// output tiles over the SMs (pairs) x per-tile time, i.e. k-blocks x the
-// measured cost of one k-block plus the part of the epilogue the variant
-// cannot overlap with the next tile.  Used only to rank the variants.
-double est_time(int impl, int64_t m, int64_t n, int kblocks, int sms) {
-  const auto waves = [](int64_t tiles, int64_t units) {
-    return static_cast<double>((tiles + units - 1) / units);
-  };
-  const double kb = kblocks;
-  switch (impl) {
-    case 1:   // 256 x 256 pair tile, one accumulator: whole epilogue exposed
-      return waves(((n + 255) / 256) * ((m + 255) / 256), sms / 2) * (0.50 * kb + 2.5);
-    case 4:   // 256 x 224 pair tile, two accumulators: only the last drain exposed
-      return waves(((n + 255) / 256) * ((m + 223) / 224), sms / 2) * std::max(0.50 * kb, 1.4) + 2.0;
-    default:  // 128 x 128 single-SM tile, two accumulators
-      return waves(((n + 127) / 128) * ((m + 127) / 128), sms) * std::max(0.48 * kb, 1.6);
-  }
-}
-
-// Tile plan.  At least 128 tokens and enough 128 x 128 tiles for half the SMs:
-// a persistent kernel, the variant with the lowest estimated time (or the
-// SP24_GEMM_IMPL override).  Otherwise (few tokens or few tiles): the split-K
-// kernel, BN from the token count and K split until the CTAs cover the SMs.
 template <int kDtype>
 sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s) {
-  const int sms = sm_count();
-  const int64_t row_tiles = (a.n + 127) / 128;
-  const bool persistent = a.m >= 128 && row_tiles * ((a.m + 127) / 128) >= sms / 2;
-  int bn = a.m <= 16 ? 16 : a.m <= 32 ? 32 : a.m <= 64 ? 64 : 128;
-  const int64_t tok_tiles = (a.m + bn - 1) / bn;
-  const int64_t base = row_tiles * tok_tiles;
-  int split = 1;
-  if (!persistent)
-    while (split < 8 && base * split < 2 * sms && a.kblocks >= 2 * split) split *= 2;
-  a.kb_per_split = (a.kblocks + split - 1) / split;
-
+  Plan p;
+  SP24_TRY(make_plan(a.m, a.n, a.kblocks, &p));
+  a.kb_per_split = (a.kblocks + p.split - 1) / p.split;
+  const int bn = p.bn;
   const int el = kDtype == SP24_BF16 ? 2 : 1;
   const CUtensorMapDataType dt =
       kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -554,34 +688,27 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
   CUtensorMap ma, mb;
   SP24_TRY(make_map(&ma, vals, dt, el, static_cast<uint64_t>(a.k / 2),
                     static_cast<uint64_t>(a.n), box_cols, 128));
+  const int pairs = static_cast<int>(p.ctas / 2);
+  switch (p.impl) {
+    case kPair256: return launch_pair_out<kDtype, 256, 4, 3, 1>(ma, a, x, pairs, s);
+    case kPair240: return launch_pair_out<kDtype, 240, 4, 3, 2>(ma, a, x, pairs, s);
+    case kPair224: return launch_pair_out<kDtype, 224, 4, 4, 2>(ma, a, x, pairs, s);
+    case kPair192: return launch_pair_out<kDtype, 192, 4, 4, 2>(ma, a, x, pairs, s);
+    case kPair128:
+      if constexpr (kDtype == SP24_BF16) {
+        return launch_pair<kDtype, 128, 6, SP24_OUT_BF16, 2>(ma, a, x, pairs, s);
+      } else {
+        if (a.out_kind == SP24_OUT_INT32)
+          return launch_pair<kDtype, 128, 5, SP24_OUT_INT32, 2>(ma, a, x, pairs, s);
+        if (a.out_kind == SP24_OUT_INT8)
+          return launch_pair<kDtype, 128, 6, SP24_OUT_INT8, 2>(ma, a, x, pairs, s);
+        return launch_pair<kDtype, 128, 5, SP24_OUT_BF16, 2>(ma, a, x, pairs, s);
+      }
+    default: break;
+  }
   SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(a.k), static_cast<uint64_t>(a.m),
                     box_cols, static_cast<uint32_t>(bn)));
-
-  if (persistent) {
-    int impl = impl_choice();
-    if (impl == 0) {
-      // pair tiles need both dimensions to fill them
-      impl = 3;
-      if (a.m >= 256 && a.n >= 256) {
-        double best = est_time(3, a.m, a.n, a.kblocks, sms);
-        for (int c : {1, 4}) {
-          const double t = est_time(c, a.m, a.n, a.kblocks, sms);
-          if (t < best) { best = t; impl = c; }
-        }
-      }
-    }
-    if (impl == 1) return launch_pair_out<kDtype, 256, 4, 3, 1>(ma, a, x, s);
-    if (impl == 4) return launch_pair_out<kDtype, 224, 4, 4, 2>(ma, a, x, s);
-    if (impl == 5) return launch_pair_out<kDtype, 192, 4, 4, 2>(ma, a, x, s);
-    if (impl == 2) {
-      if constexpr (kDtype == SP24_BF16) {
-        return launch_pair<kDtype, 128, 6, SP24_OUT_BF16, 2>(ma, a, x, s);
-      } else {
-        if (a.out_kind == SP24_OUT_INT32) return launch_pair<kDtype, 128, 5, SP24_OUT_INT32, 2>(ma, a, x, s);
-        if (a.out_kind == SP24_OUT_INT8) return launch_pair<kDtype, 128, 6, SP24_OUT_INT8, 2>(ma, a, x, s);
-        return launch_pair<kDtype, 128, 5, SP24_OUT_BF16, 2>(ma, a, x, s);
-      }
-    }
+  if (p.impl == kSingle) {
     if constexpr (kDtype == SP24_BF16) {
       return launch_persistent<kDtype, 128, 4, SP24_OUT_BF16>(ma, mb, a, s);
     } else {
@@ -590,6 +717,7 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
       return launch_persistent<kDtype, 128, 4, SP24_OUT_BF16>(ma, mb, a, s);
     }
   }
+  const int split = p.split;
 
 #define SP24_GEMM_CASE(BN_, ST_)                                                          \
   if (bn == BN_) {                                                                        \
@@ -650,4 +778,24 @@ extern "C" sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void
   a.kb_per_split = a.kblocks;
   if (dtype == SP24_BF16) return dispatch<SP24_BF16>(X, vals, a, as_stream(stream));
   return dispatch<SP24_INT8>(X, vals, a, as_stream(stream));
+}
+
+extern "C" sp24_status sp24_gemm_plan(int64_t M, int64_t N, int64_t K, int dtype,
+                                      sp24_gemm_plan_t* plan) {
+  if (!plan || M < 1 || N < 1 || K < 16 || (dtype != SP24_BF16 && dtype != SP24_INT8))
+    return SP24_ERR_ARG;
+  if (K > (int64_t(1) << 31) || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
+    return SP24_ERR_UNSUPPORTED;
+  SP24_TRY(check_device());
+  const int kl = dtype == SP24_BF16 ? 128 : 256;
+  Plan p;
+  SP24_TRY(make_plan(M, N, static_cast<int>((K + kl - 1) / kl), &p));
+  std::memset(plan, 0, sizeof(*plan));
+  std::snprintf(plan->kernel, sizeof(plan->kernel), "%s", impl_name(p.impl));
+  plan->tile_tokens = p.tile_tokens;
+  plan->tile_channels = p.tile_channels;
+  plan->split_k = p.split;
+  plan->ctas = p.ctas;
+  plan->cluster = p.cluster;
+  return SP24_OK;
 }

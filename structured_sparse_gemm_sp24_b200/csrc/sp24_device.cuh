@@ -292,6 +292,28 @@ __device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// Half of tmem_ld_16x256b_x4: 16 lanes x 16 columns into r[16*H .. 16*H + 7]
+// (register 4b + i as above, b = 0, 1).
+template <int H>
+__device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+      : "=r"(r[16 * H + 0]), "=r"(r[16 * H + 1]), "=r"(r[16 * H + 2]), "=r"(r[16 * H + 3]),
+        "=r"(r[16 * H + 4]), "=r"(r[16 * H + 5]), "=r"(r[16 * H + 6]), "=r"(r[16 * H + 7])
+      : "r"(taddr));
+}
+
+// 16 consecutive 32-bit columns of this thread's lane into r[0 .. 15].
+__device__ __forceinline__ void tmem_ld16_into(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 // Four 8x8 b16 matrices, each stored transposed: fragment element (row c, col
 // r) -- held by thread 4c + r/2 in half r&1 of register `a<m>` -- lands at
 // position c of shared row r of matrix m, whose 16-byte address thread 8m + r

@@ -64,7 +64,20 @@ SIGNATURES = {
     "sp24_last_cuda_error": (ctypes.c_char_p, []),
     "sp24_prune_wanda_noalloc": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_int, _c_p, _c_p,
                                           _c_p]),
+    "sp24_gemm_plan": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_p]),
 }
+
+
+class GemmPlan(ctypes.Structure):
+    """sp24_gemm_plan_t: the launch sp24_gemm makes for a problem."""
+    _fields_ = [("kernel", ctypes.c_char * 16), ("tile_tokens", ctypes.c_int32),
+                ("tile_channels", ctypes.c_int32), ("split_k", ctypes.c_int32),
+                ("cluster", ctypes.c_int32), ("ctas", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {"kernel": self.kernel.decode(), "tile_tokens": self.tile_tokens,
+                "tile_channels": self.tile_channels, "split_k": self.split_k,
+                "cluster": self.cluster, "ctas": self.ctas}
 
 _LIB: Optional[ctypes.CDLL] = None
 
@@ -213,6 +226,13 @@ def sp24_gemm(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, N: int, d
     _check(lib().sp24_gemm(_ptr(X), M, K, _ptr(vals), _ptr(meta), N, dtype, _ptr(s_x),
                            _ptr(s_w), out_kind, _ptr(s_y), _ptr(Y), _stream(stream)),
            "sp24_gemm")
+
+
+def sp24_gemm_plan(M: int, N: int, K: int, dtype: int) -> dict:
+    """The kernel, tile and grid sp24_gemm uses for an M x N x K problem."""
+    plan = GemmPlan()
+    _check(lib().sp24_gemm_plan(M, N, K, dtype, ctypes.byref(plan)), "sp24_gemm_plan")
+    return plan.as_dict()
 
 
 def sp24_device_status(stream=None) -> int:

@@ -424,7 +424,7 @@ def gemm_impl(request, monkeypatch):
     return request.param
 
 
-@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair256"], indirect=True)
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair240", "pair256"], indirect=True)
 @pytest.mark.parametrize("mnk", IMPL_SHAPES)
 def test_gemm_bf16_impls(gemm_impl, mnk):
     m, n, k = mnk
@@ -435,7 +435,7 @@ def test_gemm_bf16_impls(gemm_impl, mnk):
     ok_status()
 
 
-@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair256"], indirect=True)
+@pytest.mark.parametrize("gemm_impl", ["single", "pair128", "pair192", "pair224", "pair240", "pair256"], indirect=True)
 @pytest.mark.parametrize("out_kind", [B.SP24_OUT_INT32, B.SP24_OUT_BF16, B.SP24_OUT_INT8])
 @pytest.mark.parametrize("mnk", [(2500, 2064, 416), (130, 528, 96 + 32), (3000, 1808, 1280)])
 def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
@@ -452,3 +452,24 @@ def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
     else:
         assert np.array_equal(y.cpu().numpy(), O.requant_int8(acc, s_x, s_w, np.float32(0.05)))
     ok_status()
+
+
+# ------------------------------------------------------------ launch plans
+def test_gemm_plan_families(monkeypatch):
+    monkeypatch.delenv("SP24_GEMM_IMPL", raising=False)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    small = B.sp24_gemm_plan(16, 11008, 4096, B.SP24_BF16)
+    assert small["kernel"] == "splitk" and small["tile_tokens"] == 16
+    assert small["split_k"] >= 1 and small["cluster"] == small["split_k"]
+    big = B.sp24_gemm_plan(8192, 8192, 8192, B.SP24_BF16)
+    assert big["kernel"].startswith("pair") and big["cluster"] == 2
+    # a persistent pair grid never exceeds the resident pairs (<= SMs / 2)
+    assert big["ctas"] % 2 == 0 and 2 <= big["ctas"] <= sms
+    conv = B.sp24_gemm_plan(200704, 64, 256, B.SP24_BF16)
+    assert conv["kernel"] == "single" and conv["ctas"] == sms
+    monkeypatch.setenv("SP24_GEMM_IMPL", "pair240")
+    forced = B.sp24_gemm_plan(4096, 3072, 768, B.SP24_BF16)
+    assert forced["kernel"] == "pair240" and forced["tile_tokens"] == 240
+    assert forced["tile_channels"] == 256
+    with pytest.raises(B.Sp24Error):
+        B.sp24_gemm_plan(0, 64, 64, B.SP24_BF16)
