@@ -527,21 +527,219 @@ __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict_
 }
 
 // ----------------------------------------------------- a5 activation scale
-// Exact radix selection of the r-th smallest |x| over a float32 tensor:
-// keys = bits & 0x7FFFFFFF (monotone in |x| for finite x), three passes of
-// 11/11/9 bits.  Workspace: 2048 histogram counters + {prefix, rank}.
+// Exact selection of the r-th smallest |x| over a float32 tensor, on keys =
+// bits & 0x7FFFFFFF (monotone in |x| for finite x).
+//
+// Fast path (large tensors), exact whenever it reports success:
+//  1. act_sample: one CTA takes kActSample keys at stratified, hashed
+//     positions and selects two order statistics of the sample around the
+//     sample rank of r (six standard deviations of a binomial count on each
+//     side): the bracket [lo, hi].
+//  2. act_bracket: one pass over the tensor counts keys < lo and appends the
+//     keys in [lo, hi] to a candidate list.
+//  3. act_bracket_select: if  below < r <= below + candidates  (and the list
+//     did not overflow) the answer is the (r - below)-th smallest candidate,
+//     selected exactly; otherwise nothing is decided.
+// Fallback (small tensors, or a bracket that missed): three radix passes of
+// 11/11/9 bits over the whole tensor; every fallback kernel returns at once
+// when the fast path already decided.
+constexpr int kActSample = 16384;
+constexpr uint32_t kActCandCap = 1u << 20;
+constexpr int64_t kActBracketMin = int64_t(1) << 18;   // smaller tensors: radix only
+
 struct ActScaleWs {
-  uint32_t hist[2048];
-  uint32_t prefix;   // selected high bits so far
-  uint32_t rank;     // remaining 1-based rank within the current prefix
-  uint32_t pad[2];
+  uint32_t hist[2048];   // radix histogram
+  uint32_t prefix;       // radix: selected high bits so far
+  uint32_t rank;         // radix: remaining 1-based rank within the prefix
+  uint32_t lo, hi;       // bracket keys (inclusive)
+  uint32_t below;        // keys < lo
+  uint32_t ncand;        // keys in [lo, hi] (counts past the capacity)
+  uint32_t done;         // 1 once s_x holds the answer
+  uint32_t pad;
+  uint32_t cand[kActCandCap];
 };
+
+// Inclusive prefix sum of v over a block of 1024 threads (scratch: 32 words).
+__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) scratch[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = scratch[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    scratch[lane] = w;
+  }
+  __syncthreads();
+  if (warp > 0) v += scratch[warp - 1];
+  __syncthreads();
+  return v;
+}
+
+// k-th smallest (1-based; 1 <= k <= n) of the n keys key_at(0 .. n-1), by a
+// block of 1024 threads: three radix passes of 11/11/9 bits over a shared
+// histogram.  hist: 2048 words; scratch: 34 words.
+template <class KeyAt>
+__device__ uint32_t block_select(KeyAt key_at, uint32_t n, uint32_t k, uint32_t* hist,
+                                 uint32_t* scratch) {
+  const int shifts[3] = {20, 9, 0};
+  const int bitsv[3] = {11, 11, 9};
+  uint32_t prefix = 0, mask = 0;
+  for (int p = 0; p < 3; ++p) {
+    const uint32_t nb = 1u << bitsv[p];
+    for (uint32_t i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t key = key_at(i);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shifts[p]) & (nb - 1u)], 1u);
+    }
+    __syncthreads();
+    const uint32_t b0 = 2u * threadIdx.x;
+    const uint32_t h0 = b0 < nb ? hist[b0] : 0u;
+    const uint32_t h1 = b0 + 1u < nb ? hist[b0 + 1u] : 0u;
+    const uint32_t incl = block_incl_scan(h0 + h1, scratch);
+    const uint32_t excl = incl - h0 - h1;
+    if (excl < k && k <= incl) {   // exactly one thread holds the k-th key's bin
+      const bool second = k > excl + h0;
+      scratch[32] = b0 + (second ? 1u : 0u);
+      scratch[33] = excl + (second ? h0 : 0u);
+    }
+    __syncthreads();
+    const uint32_t bin = scratch[32], below = scratch[33];
+    __syncthreads();
+    prefix |= bin << shifts[p];
+    mask |= (nb - 1u) << shifts[p];
+    k -= below;
+  }
+  return prefix;
+}
+
+__device__ __forceinline__ uint32_t abs_key(float v) { return __float_as_uint(v) & 0x7FFFFFFFu; }
+
+__device__ __forceinline__ uint32_t mix32(uint32_t v) {   // integer hash (xorshift-multiply)
+  v ^= v >> 16;
+  v *= 0x7feb352du;
+  v ^= v >> 15;
+  v *= 0x846ca68bu;
+  v ^= v >> 16;
+  return v;
+}
 
 __global__ void act_scale_init(ActScaleWs* ws, uint32_t rank) {
   for (int i = threadIdx.x; i < 2048; i += blockDim.x) ws->hist[i] = 0;
   if (threadIdx.x == 0) {
     ws->prefix = 0;
     ws->rank = rank;
+    ws->done = 0;
+  }
+}
+
+// Dynamic shared memory: kActSample keys.
+__global__ void __launch_bounds__(1024) act_sample(const float* __restrict__ x, int64_t count,
+                                                   uint32_t rank, ActScaleWs* ws) {
+  extern __shared__ uint32_t keys[];
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t scratch[34];
+  const int64_t stride = count / kActSample;   // >= 16 (count >= kActBracketMin)
+  for (int i = threadIdx.x; i < kActSample; i += blockDim.x) {
+    const int64_t pos = static_cast<int64_t>(i) * stride +
+                        static_cast<int64_t>(mix32(static_cast<uint32_t>(i)) % stride);
+    keys[i] = abs_key(__ldg(x + pos));
+  }
+  for (int i = threadIdx.x; i < 2048; i += blockDim.x) ws->hist[i] = 0;
+  __syncthreads();
+  const double q = static_cast<double>(rank) / static_cast<double>(count);
+  const double sd = sqrt(static_cast<double>(kActSample) * q * (1.0 - q));
+  const int64_t half = static_cast<int64_t>(ceil(6.0 * sd)) + 4;
+  int64_t rs = static_cast<int64_t>(ceil(q * kActSample));
+  rs = rs < 1 ? 1 : (rs > kActSample ? kActSample : rs);
+  const auto at = [&](uint32_t i) { return keys[i]; };
+  const uint32_t lo = rs - half >= 1
+      ? block_select(at, kActSample, static_cast<uint32_t>(rs - half), hist, scratch) : 0u;
+  const uint32_t hi = rs + half <= kActSample
+      ? block_select(at, kActSample, static_cast<uint32_t>(rs + half), hist, scratch)
+      : 0xFFFFFFFFu;
+  if (threadIdx.x == 0) {
+    ws->lo = lo;
+    ws->hi = hi;
+    ws->below = 0;
+    ws->ncand = 0;
+    ws->done = 0;
+    ws->prefix = 0;
+    ws->rank = rank;
+  }
+}
+
+__device__ __forceinline__ void bracket_one(uint32_t key, bool valid, uint32_t lo, uint32_t hi,
+                                            uint32_t& below, ActScaleWs* ws, int lane) {
+  below += (valid && key < lo) ? 1u : 0u;
+  const bool c = valid && key >= lo && key <= hi;
+  const uint32_t m = __ballot_sync(0xffffffffu, c);
+  if (m) {
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if (lane == leader) base = atomicAdd(&ws->ncand, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (c) {
+      const uint32_t idx = base + __popc(m & ((1u << lane) - 1u));
+      if (idx < kActCandCap) ws->cand[idx] = key;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x, int64_t nvec,
+                                                   const float* __restrict__ tail, int ntail,
+                                                   ActScaleWs* ws) {
+  __shared__ uint32_t part[8];
+  const uint32_t lo = ws->lo, hi = ws->hi;
+  const int lane = threadIdx.x & 31;
+  uint32_t below = 0;
+  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  for (int64_t base = gw * 32; base < nvec; base += warps * 32) {   // warp-uniform trip count
+    const int64_t v = base + lane;
+    const bool valid = v < nvec;
+    const float4 q = valid ? __ldcs(x + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+    bracket_one(abs_key(q.x), valid, lo, hi, below, ws, lane);
+    bracket_one(abs_key(q.y), valid, lo, hi, below, ws, lane);
+    bracket_one(abs_key(q.z), valid, lo, hi, below, ws, lane);
+    bracket_one(abs_key(q.w), valid, lo, hi, below, ws, lane);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    const bool valid = lane < ntail;
+    bracket_one(valid ? abs_key(tail[lane]) : 0u, valid, lo, hi, below, ws, lane);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+  if (lane == 0) part[threadIdx.x >> 5] = below;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t t = 0;
+    for (int w = 0; w < (blockDim.x >> 5); ++w) t += part[w];
+    if (t) atomicAdd(&ws->below, t);
+  }
+}
+
+__global__ void __launch_bounds__(1024) act_bracket_select(ActScaleWs* ws, float* s_x) {
+  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t scratch[34];
+  const uint32_t below = ws->below, n = ws->ncand, rank = ws->rank;
+  if (!(below < rank && rank - below <= n && n <= kActCandCap)) return;   // radix decides
+  const uint32_t* cand = ws->cand;
+  const uint32_t key =
+      block_select([&](uint32_t i) { return cand[i]; }, n, rank - below, hist, scratch);
+  if (threadIdx.x == 0) {
+    const float t = __uint_as_float(key);
+    *s_x = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
+    ws->done = 1;
   }
 }
 
@@ -549,6 +747,7 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
                                                       const float* __restrict__ tail,
                                                       int ntail, ActScaleWs* ws, int shift,
                                                       int bits, uint32_t hi_mask) {
+  if (ws->done) return;
   __shared__ uint32_t h[2048];
   const uint32_t nb = 1u << bits;
   for (uint32_t i = threadIdx.x; i < nb; i += blockDim.x) h[i] = 0;
@@ -561,13 +760,13 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
     const float e[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint32_t key = __float_as_uint(e[i]) & 0x7FFFFFFFu;
+      const uint32_t key = abs_key(e[i]);
       if ((key & hi_mask) == prefix) atomicAdd(&h[(key >> shift) & (nb - 1u)], 1u);
     }
   }
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < ntail; i += blockDim.x) {
-      const uint32_t key = __float_as_uint(tail[i]) & 0x7FFFFFFFu;
+      const uint32_t key = abs_key(tail[i]);
       if ((key & hi_mask) == prefix) atomicAdd(&h[(key >> shift) & (nb - 1u)], 1u);
     }
   }
@@ -577,7 +776,7 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
 }
 
 __global__ void act_scale_select(ActScaleWs* ws, int shift, int bits, float* s_x, int last) {
-  if (threadIdx.x != 0) return;
+  if (threadIdx.x != 0 || ws->done) return;
   const uint32_t nb = 1u << bits;
   uint32_t below = 0, b = 0;
   for (b = 0; b < nb - 1u; ++b) {
@@ -817,10 +1016,31 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
   uint32_t rank = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
   if (rank > static_cast<uint64_t>(count)) rank = static_cast<uint32_t>(count);
   ActScaleWs* ws = static_cast<ActScaleWs*>(workspace);
-  act_scale_init<<<1, 256, 0, s>>>(ws, rank);
-  SP24_TRY(launch_status());
   const int64_t nvec = count / 4;
   const int ntail = static_cast<int>(count - nvec * 4);
+  if (count >= kActBracketMin) {
+    static uint64_t attr_set = 0;   // one bit per device (devices 0..63)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+    const uint64_t bit = 1ull << (dev & 63);
+    const int sample_smem = kActSample * 4;
+    if (!(attr_set & bit)) {
+      const cudaError_t e = cudaFuncSetAttribute(
+          act_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, sample_smem);
+      if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+      attr_set |= bit;
+    }
+    act_sample<<<1, 1024, sample_smem, s>>>(X, count, rank, ws);
+    SP24_TRY(launch_status());
+    act_bracket<<<grid_for(nvec, 256), 256, 0, s>>>(reinterpret_cast<const float4*>(X), nvec,
+                                                     X + nvec * 4, ntail, ws);
+    SP24_TRY(launch_status());
+    act_bracket_select<<<1, 1024, 0, s>>>(ws, s_x);
+    SP24_TRY(launch_status());
+  } else {
+    act_scale_init<<<1, 256, 0, s>>>(ws, rank);
+    SP24_TRY(launch_status());
+  }
   const int grid = grid_for(nvec, 256);
   const int shifts[3] = {20, 9, 0};
   const int bitsv[3] = {11, 11, 9};

@@ -236,6 +236,32 @@ def test_act_scale_and_quantize_small(count):
     assert np.array_equal(q.cpu().numpy(), O.quantize(x.numpy(), rs))
 
 
+def _act_inputs(kind, count, seed):
+    x = I.normal_f32((count,), 1.0, seed=seed).numpy()
+    if kind == "ties":          # coarse values: thousands of equal keys at the quantile
+        x = np.round(x * 4.0) / 4.0
+    elif kind == "outlier_cols":  # a few "channels" of a 1024-wide matrix carry x50 outliers
+        body = x[: (count // 1024) * 1024].reshape(-1, 1024)   # a view into x
+        body[:, [3, 517, 1000]] *= 50.0
+    elif kind == "zeros":       # mostly exact zeros (ReLU-like), a sparse positive tail
+        x = np.where(x > 2.5, x, 0.0).astype(np.float32)
+    elif kind == "constant":    # one key everywhere but 8 outliers: more equal candidates
+        x = np.full(count, 0.75, dtype=np.float32)   # than the bracket list holds, so the
+        x[np.arange(8) * (count // 8)] = 9.0          # exact radix fallback decides
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+
+
+@pytest.mark.parametrize("kind", ["normal", "ties", "outlier_cols", "zeros", "constant"])
+@pytest.mark.parametrize("coverage", [0.5, 0.9, 0.9999, 1.0])
+def test_act_scale_large_coverages(kind, coverage):
+    # >= 2^18 elements take the sampled-bracket path; central coverages, heavy
+    # ties and column-structured outliers exercise its exact fallback
+    x = _act_inputs(kind, (1 << 20) + 12, seed=77)
+    s = P.act_scale(x.cuda(), coverage)
+    assert s.item() == O.tensor_scale(x.numpy(), coverage)
+    ok_status()
+
+
 def test_act_scale_and_quantize_int8_workload():
     w = I.int8_long_tail()
     xd = w.X.cuda()
