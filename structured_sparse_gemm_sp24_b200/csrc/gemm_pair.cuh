@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
              const __grid_constant__ CUtensorMap tmap_y16, const PersistArgs args) {
+  pdl_launch_dependents();
   using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -105,6 +106,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   cluster_sync();          // barriers of both CTAs initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_prior();   // set-up above overlapped the previous kernel's tail
 
   if (warp == 0) {
     if (lane == 0) {

@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,
                    const __grid_constant__ CUtensorMap tmap_y, const PersistArgs args) {
+  pdl_launch_dependents();
   using C = PersistCfg<kDtype, BN, STAGES, OUTK>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -108,6 +109,7 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_prior();   // set-up above overlapped the previous kernel's tail
   const int kchunks = static_cast<int>((args.k + 127) / 128);
 
   if (warp == 0) {

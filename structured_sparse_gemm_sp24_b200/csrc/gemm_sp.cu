@@ -93,6 +93,8 @@ template <int kDtype, int BN, int STAGES, int SPLIT>
 __global__ void __launch_bounds__(128, 1)
 gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
                const __grid_constant__ CUtensorMap tmap_b, const GemmArgs args) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   using C = GemmCfg<kDtype, BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -344,21 +346,9 @@ sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const 
   const int64_t row_tiles = (a.n + 127) / 128;
   const int64_t tok_tiles = (a.m + BN - 1) / BN;
   if (row_tiles > 65535 || tok_tiles > 65535) return SP24_ERR_UNSUPPORTED;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(SPLIT, static_cast<unsigned>(row_tiles), static_cast<unsigned>(tok_tiles));
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = SPLIT;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, a);
-  if (le != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", le);
-  return launch_status();
+  return launch_kernel(kern, dim3(SPLIT, static_cast<unsigned>(row_tiles),
+                                  static_cast<unsigned>(tok_tiles)),
+                       dim3(128), C::kSmemBytes, s, SPLIT, ma, mb, a);
 }
 
 
@@ -405,8 +395,8 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
   const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
   if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
   const int grid = static_cast<int>(ntiles < sm_count() ? ntiles : sm_count());
-  kern<<<grid, 64 + kEpiThreads, C::kSmemBytes, s>>>(ma, mb, my, a);
-  return launch_status();
+  return launch_kernel(kern, dim3(grid), dim3(64 + kEpiThreads), C::kSmemBytes, s, 1, ma, mb, my,
+                       a);
 }
 
 
@@ -474,21 +464,8 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
   if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
   if (pairs < 1 || pairs > ntiles) return SP24_ERR_ARG;   // the plan sizes the grid
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(64 + kEpiThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, kern, ma, mb, me, my, my16, a);
-  if (le != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", le);
-  return launch_status();
+  return launch_kernel(kern, dim3(2 * pairs), dim3(64 + kEpiThreads), C::kSmemBytes, s, 2, ma,
+                       mb, me, my, my16, a);
 }
 
 // Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair240 |

@@ -151,6 +151,8 @@ __device__ __forceinline__ uint32_t gather_pair(uint32_t w0, uint32_t w1, uint32
 __global__ void __launch_bounds__(256) colnorm_kernel(const uint16_t* __restrict__ xc,
                                                       int64_t mc, int64_t k,
                                                       double* __restrict__ norms) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   __shared__ __align__(16) uint16_t tile[128][64];
   const int64_t col0 = static_cast<int64_t>(blockIdx.x) * 64;
   const int cvalid = static_cast<int>(k - col0 < 64 ? k - col0 : 64);   // multiple of 8
@@ -249,6 +251,8 @@ __global__ void __launch_bounds__(kStreamThreads, 1)
 stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_mask,
               const __grid_constant__ CUtensorMap tm_norm, const __grid_constant__ CUtensorMap tm_sw,
               const StreamArgs a) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -448,6 +452,8 @@ __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict_
                                                      const uint8_t* __restrict__ mask, int64_t n,
                                                      int64_t k, double coverage,
                                                      float* __restrict__ s_w) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   __shared__ uint32_t hist[8][256];
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t wid = threadIdx.x >> 5;
@@ -634,6 +640,8 @@ __device__ __forceinline__ uint32_t mix32(uint32_t v) {   // integer hash (xorsh
 }
 
 __global__ void act_scale_init(ActScaleWs* ws, uint32_t rank) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   for (int i = threadIdx.x; i < 2048; i += blockDim.x) ws->hist[i] = 0;
   if (threadIdx.x == 0) {
     ws->prefix = 0;
@@ -645,6 +653,8 @@ __global__ void act_scale_init(ActScaleWs* ws, uint32_t rank) {
 // Dynamic shared memory: kActSample keys.
 __global__ void __launch_bounds__(1024) act_sample(const float* __restrict__ x, int64_t count,
                                                    uint32_t rank, ActScaleWs* ws) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   extern __shared__ uint32_t keys[];
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t scratch[34];
@@ -698,6 +708,8 @@ __device__ __forceinline__ void bracket_one(uint32_t key, bool valid, uint32_t l
 __global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x, int64_t nvec,
                                                    const float* __restrict__ tail, int ntail,
                                                    ActScaleWs* ws) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   __shared__ uint32_t part[8];
   const uint32_t lo = ws->lo, hi = ws->hi;
   const int lane = threadIdx.x & 31;
@@ -729,6 +741,8 @@ __global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x,
 }
 
 __global__ void __launch_bounds__(1024) act_bracket_select(ActScaleWs* ws, float* s_x) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t scratch[34];
   const uint32_t below = ws->below, n = ws->ncand, rank = ws->rank;
@@ -747,6 +761,8 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
                                                       const float* __restrict__ tail,
                                                       int ntail, ActScaleWs* ws, int shift,
                                                       int bits, uint32_t hi_mask) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   if (ws->done) return;
   __shared__ uint32_t h[2048];
   const uint32_t nb = 1u << bits;
@@ -776,6 +792,8 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
 }
 
 __global__ void act_scale_select(ActScaleWs* ws, int shift, int bits, float* s_x, int last) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   if (threadIdx.x != 0 || ws->done) return;
   const uint32_t nb = 1u << bits;
   uint32_t below = 0, b = 0;
@@ -802,6 +820,8 @@ __device__ __forceinline__ uint32_t q8(float x, float s) {
 __global__ void __launch_bounds__(256) quantize_kernel(const float4* __restrict__ x, int64_t nvec16,
                                                        const float* __restrict__ s_ptr,
                                                        uint4* __restrict__ xq) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   const float s = *s_ptr;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec16;
@@ -818,6 +838,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float4* __restrict_
 
 __global__ void quantize_tail(const float* __restrict__ x, int64_t start, int64_t count,
                               const float* __restrict__ s_ptr, int8_t* __restrict__ xq) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   const int64_t i = start + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i < count) xq[i] = static_cast<int8_t>(q8(x[i], *s_ptr));
 }
@@ -865,8 +887,8 @@ static int grid_for(int64_t work_items, int threads) {
 static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double* norms,
                                   cudaStream_t s) {
   const int blocks = static_cast<int>((k + 63) / 64);
-  colnorm_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint16_t*>(xc), mc, k, norms);
-  return launch_status();
+  return launch_kernel(colnorm_kernel, dim3(blocks), dim3(256), 0, s, 1,
+                       static_cast<const uint16_t*>(xc), mc, k, norms);
 }
 
 template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
@@ -916,8 +938,8 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
   a.vals = vals;
   a.meta = static_cast<uint8_t*>(meta);
   const int grid = static_cast<int>(nchunks < sm_count() ? nchunks : sm_count());
-  kern<<<grid, kStreamThreads, kStreamSmem, s>>>(tw, tm, tn, ts, a);
-  return launch_status();
+  return launch_kernel(kern, dim3(grid), dim3(kStreamThreads), kStreamSmem, s, 1, tw, tm, tn, ts,
+                       a);
 }
 
 // For the pruning variants `mask` is mask_in (optional); a separate
@@ -997,9 +1019,9 @@ sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K
   if (K % 8 != 0 || !aligned16(W) || !aligned16(mask) || !aligned16(s_w)) return SP24_ERR_ALIGN;
   if (N > 0x7FFFFFFF) return SP24_ERR_ARG;
   SP24_TRY(check_device());
-  wscale_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, as_stream(stream)>>>(
-      static_cast<const uint16_t*>(W), mask, N, K, coverage, s_w);
-  return launch_status();
+  return launch_kernel(wscale_kernel, dim3(static_cast<unsigned>((N + 7) / 8)), dim3(256), 0,
+                       as_stream(stream), 1, static_cast<const uint16_t*>(W), mask, N, K,
+                       coverage, s_w);
 }
 
 size_t sp24_act_scale_workspace_bytes(void) { return sizeof(ActScaleWs); }
@@ -1030,27 +1052,24 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
       if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
       attr_set |= bit;
     }
-    act_sample<<<1, 1024, sample_smem, s>>>(X, count, rank, ws);
-    SP24_TRY(launch_status());
-    act_bracket<<<grid_for(nvec, 256), 256, 0, s>>>(reinterpret_cast<const float4*>(X), nvec,
-                                                     X + nvec * 4, ntail, ws);
-    SP24_TRY(launch_status());
-    act_bracket_select<<<1, 1024, 0, s>>>(ws, s_x);
-    SP24_TRY(launch_status());
+    SP24_TRY(launch_kernel(act_sample, dim3(1), dim3(1024), sample_smem, s, 1, X, count, rank,
+                           ws));
+    SP24_TRY(launch_kernel(act_bracket, dim3(grid_for(nvec, 256)), dim3(256), 0, s, 1,
+                           reinterpret_cast<const float4*>(X), nvec, X + nvec * 4, ntail, ws));
+    SP24_TRY(launch_kernel(act_bracket_select, dim3(1), dim3(1024), 0, s, 1, ws, s_x));
   } else {
-    act_scale_init<<<1, 256, 0, s>>>(ws, rank);
-    SP24_TRY(launch_status());
+    SP24_TRY(launch_kernel(act_scale_init, dim3(1), dim3(256), 0, s, 1, ws, rank));
   }
   const int grid = grid_for(nvec, 256);
   const int shifts[3] = {20, 9, 0};
   const int bitsv[3] = {11, 11, 9};
   uint32_t hi_mask = 0;
   for (int p = 0; p < 3; ++p) {
-    act_scale_hist<<<grid, 256, 0, s>>>(reinterpret_cast<const float4*>(X), nvec,
-                                        X + nvec * 4, ntail, ws, shifts[p], bitsv[p], hi_mask);
-    SP24_TRY(launch_status());
-    act_scale_select<<<1, 32, 0, s>>>(ws, shifts[p], bitsv[p], s_x, p == 2);
-    SP24_TRY(launch_status());
+    SP24_TRY(launch_kernel(act_scale_hist, dim3(grid), dim3(256), 0, s, 1,
+                           reinterpret_cast<const float4*>(X), nvec, X + nvec * 4, ntail, ws,
+                           shifts[p], bitsv[p], hi_mask));
+    SP24_TRY(launch_kernel(act_scale_select, dim3(1), dim3(32), 0, s, 1, ws, shifts[p],
+                           bitsv[p], s_x, static_cast<int>(p == 2)));
     hi_mask |= ((1u << bitsv[p]) - 1u) << shifts[p];
   }
   return SP24_OK;
@@ -1066,15 +1085,13 @@ sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x, int8_
   cudaStream_t s = as_stream(stream);
   const int64_t nvec16 = count / 16;
   if (nvec16 > 0) {
-    quantize_kernel<<<grid_for(nvec16, 256), 256, 0, s>>>(reinterpret_cast<const float4*>(X),
-                                                         nvec16, s_x,
-                                                         reinterpret_cast<uint4*>(Xq));
-    SP24_TRY(launch_status());
+    SP24_TRY(launch_kernel(quantize_kernel, dim3(grid_for(nvec16, 256)), dim3(256), 0, s, 1,
+                           reinterpret_cast<const float4*>(X), nvec16, s_x,
+                           reinterpret_cast<uint4*>(Xq)));
   }
   const int64_t start = nvec16 * 16;
   if (start < count) {
-    quantize_tail<<<1, 32, 0, s>>>(X, start, count, s_x, Xq);
-    SP24_TRY(launch_status());
+    SP24_TRY(launch_kernel(quantize_tail, dim3(1), dim3(32), 0, s, 1, X, start, count, s_x, Xq));
   }
   return SP24_OK;
 }

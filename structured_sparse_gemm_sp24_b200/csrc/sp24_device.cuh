@@ -30,6 +30,18 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  Every kernel of the library calls
+// pdl_launch_dependents() on entry (the next kernel of the stream may then be
+// scheduled and run its set-up) and pdl_wait_prior() before its first
+// global-memory access (blocks until the previous kernel of the stream has
+// completed and its memory operations are visible).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_prior() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

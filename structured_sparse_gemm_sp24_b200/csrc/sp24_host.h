@@ -34,6 +34,38 @@ inline sp24_status launch_status() {
 // Number of SMs of the current device (cached).
 int sm_count();
 
+// Launches every kernel of the library: programmatic stream serialization
+// (the kernel may be scheduled while the previous kernel of the stream is
+// finishing; each kernel of this library executes griddepcontrol.wait before
+// it touches global memory, so it still sees all of that kernel's results)
+// and, for cluster > 1, clusters of `cluster` CTAs along x.
+template <class... KArgs, class... Args>
+sp24_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t s, unsigned cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return cuda_fail("cudaLaunchKernelEx", e);
+  return launch_status();
+}
+
 }  // namespace sp24
 
 #define SP24_TRY(expr)                    \
