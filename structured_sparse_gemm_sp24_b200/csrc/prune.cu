@@ -159,11 +159,20 @@ __global__ void __launch_bounds__(256) colnorm_kernel(const uint16_t* __restrict
   double acc = 0.0;
   for (int64_t t0 = 0; t0 < mc; t0 += 128) {
     const int rows = static_cast<int>(mc - t0 < 128 ? mc - t0 : 128);
-    for (int i = threadIdx.x; i < rows * 8; i += blockDim.x) {
+    // 128 x 8 16-byte pieces, four per thread, all loads issued before the stores
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = threadIdx.x + u * 256;
       const int r = i >> 3, c8 = (i & 7) * 8;
-      if (c8 < cvalid)
-        *reinterpret_cast<uint4*>(&tile[r][c8]) =
-            __ldg(reinterpret_cast<const uint4*>(xc + (t0 + r) * k + col0 + c8));
+      if (r < rows && c8 < cvalid)
+        v[u] = __ldg(reinterpret_cast<const uint4*>(xc + (t0 + r) * k + col0 + c8));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = threadIdx.x + u * 256;
+      const int r = i >> 3, c8 = (i & 7) * 8;
+      if (r < rows && c8 < cvalid) *reinterpret_cast<uint4*>(&tile[r][c8]) = v[u];
     }
     __syncthreads();
     if (threadIdx.x < cvalid) {
@@ -537,10 +546,10 @@ __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict_
 // bits & 0x7FFFFFFF (monotone in |x| for finite x).
 //
 // Fast path (large tensors), exact whenever it reports success:
-//  1. act_sample: one CTA takes kActSample keys at stratified, hashed
-//     positions and selects two order statistics of the sample around the
-//     sample rank of r (six standard deviations of a binomial count on each
-//     side): the bracket [lo, hi].
+//  1. act_sample_load / act_sample_select: a histogram of kActSample keys at
+//     stratified, hashed positions; the histogram bins around the sample rank
+//     of r (six standard deviations of a binomial count on each side) give
+//     the bracket [lo, hi].
 //  2. act_bracket: one pass over the tensor counts keys < lo and appends the
 //     keys in [lo, hi] to a candidate list.
 //  3. act_bracket_select: if  below < r <= below + candidates  (and the list
@@ -561,7 +570,7 @@ struct ActScaleWs {
   uint32_t below;        // keys < lo
   uint32_t ncand;        // keys in [lo, hi] (counts past the capacity)
   uint32_t done;         // 1 once s_x holds the answer
-  uint32_t pad;
+  uint32_t blocks_done;  // radix pass: CTAs finished (the last one selects)
   uint32_t cand[kActCandCap];
 };
 
@@ -591,21 +600,23 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* scratc
 }
 
 // k-th smallest (1-based; 1 <= k <= n) of the n keys key_at(0 .. n-1), by a
-// block of 1024 threads: three radix passes of 11/11/9 bits over a shared
-// histogram.  hist: 2048 words; scratch: 34 words.
+// block of 1024 threads: radix passes of up to 11 bits over a shared
+// histogram, from bit top-1 down to bit 0.  All keys must agree with `fixed`
+// on the bits at and above `top` (for unconstrained 31-bit keys: top = 31,
+// fixed = 0).  hist: 2048 words; scratch: 34 words.
 template <class KeyAt>
 __device__ uint32_t block_select(KeyAt key_at, uint32_t n, uint32_t k, uint32_t* hist,
-                                 uint32_t* scratch) {
-  const int shifts[3] = {20, 9, 0};
-  const int bitsv[3] = {11, 11, 9};
-  uint32_t prefix = 0, mask = 0;
-  for (int p = 0; p < 3; ++p) {
-    const uint32_t nb = 1u << bitsv[p];
+                                 uint32_t* scratch, int top = 31, uint32_t fixed = 0) {
+  uint32_t prefix = top >= 31 ? 0u : (fixed & ~((1u << top) - 1u));
+  uint32_t mask = top >= 31 ? 0u : (0x7FFFFFFFu & ~((1u << top) - 1u));
+  while (top > 0) {
+    const int shift = top > 11 ? top - 11 : 0;
+    const uint32_t nb = 1u << (top - shift);
     for (uint32_t i = threadIdx.x; i < 2048; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     for (uint32_t i = threadIdx.x; i < n; i += blockDim.x) {
       const uint32_t key = key_at(i);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shifts[p]) & (nb - 1u)], 1u);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1u)], 1u);
     }
     __syncthreads();
     const uint32_t b0 = 2u * threadIdx.x;
@@ -621,9 +632,10 @@ __device__ uint32_t block_select(KeyAt key_at, uint32_t n, uint32_t k, uint32_t*
     __syncthreads();
     const uint32_t bin = scratch[32], below = scratch[33];
     __syncthreads();
-    prefix |= bin << shifts[p];
-    mask |= (nb - 1u) << shifts[p];
+    prefix |= bin << shift;
+    mask |= (nb - 1u) << shift;
     k -= below;
+    top = shift;
   }
   return prefix;
 }
@@ -647,109 +659,204 @@ __global__ void act_scale_init(ActScaleWs* ws, uint32_t rank) {
     ws->prefix = 0;
     ws->rank = rank;
     ws->done = 0;
+    ws->blocks_done = 0;
   }
 }
 
-// Dynamic shared memory: kActSample keys.
-__global__ void __launch_bounds__(1024) act_sample(const float* __restrict__ x, int64_t count,
-                                                   uint32_t rank, ActScaleWs* ws) {
+// Sample: kActSample keys at stratified, hashed positions (stratum i =
+// [i * stride, (i + 1) * stride), stride = count / kActSample in [16, 2^17],
+// offset = a hash of i scaled to the stratum), one per thread of
+// kActSampleCtas CTAs so that the scattered loads spread over many SMs.  Each
+// CTA writes the histogram of its keys' top 11 bits (bits 30..20: exponent
+// and 3 mantissa bits) to its own 2048-word slice at the start of the
+// candidate list (which act_bracket overwrites afterwards).
+constexpr int kActSampleCtas = kActSample / 1024;
+
+__global__ void __launch_bounds__(1024) act_sample_load(const float* __restrict__ x,
+                                                        int64_t count, ActScaleWs* ws) {
   pdl_launch_dependents();
   pdl_wait_prior();
-  extern __shared__ uint32_t keys[];
-  __shared__ uint32_t hist[2048];
+  __shared__ uint32_t h[2048];
+  h[threadIdx.x] = 0;
+  h[threadIdx.x + 1024] = 0;
+  __syncthreads();
+  const uint32_t stride = static_cast<uint32_t>(count / kActSample);
+  const uint32_t i = blockIdx.x * 1024u + threadIdx.x;
+  const uint32_t off = __umulhi(mix32(i), stride);
+  const uint32_t key = abs_key(__ldg(x + (static_cast<int64_t>(i) * stride + off)));
+  atomicAdd(&h[key >> 20], 1u);
+  __syncthreads();
+  uint32_t* out = ws->cand + blockIdx.x * 2048u;
+  out[threadIdx.x] = h[threadIdx.x];
+  out[threadIdx.x + 1024] = h[threadIdx.x + 1024];
+}
+
+// Sums the per-CTA sample histograms and brackets the target: lo = lower edge
+// of the bin holding sample rank rs - half, hi = upper edge of the bin holding
+// rs + half (six binomial standard deviations of the sample count on each
+// side; 0 / all-ones when the rank falls off the sample).  The bracket only
+// has to be likely: act_bracket_select checks it exactly.
+__global__ void __launch_bounds__(1024) act_sample_select(int64_t count, uint32_t rank,
+                                                          ActScaleWs* ws) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
   __shared__ uint32_t scratch[34];
-  const int64_t stride = count / kActSample;   // >= 16 (count >= kActBracketMin)
-  for (int i = threadIdx.x; i < kActSample; i += blockDim.x) {
-    const int64_t pos = static_cast<int64_t>(i) * stride +
-                        static_cast<int64_t>(mix32(static_cast<uint32_t>(i)) % stride);
-    keys[i] = abs_key(__ldg(x + pos));
+  __shared__ uint32_t bins[2];
+  const uint32_t b0 = 2u * threadIdx.x;
+  uint32_t h0 = 0, h1 = 0;
+#pragma unroll
+  for (int c = 0; c < kActSampleCtas; ++c) {
+    h0 += __ldcg(ws->cand + c * 2048 + b0);
+    h1 += __ldcg(ws->cand + c * 2048 + b0 + 1);
   }
   for (int i = threadIdx.x; i < 2048; i += blockDim.x) ws->hist[i] = 0;
-  __syncthreads();
   const double q = static_cast<double>(rank) / static_cast<double>(count);
   const double sd = sqrt(static_cast<double>(kActSample) * q * (1.0 - q));
   const int64_t half = static_cast<int64_t>(ceil(6.0 * sd)) + 4;
   int64_t rs = static_cast<int64_t>(ceil(q * kActSample));
   rs = rs < 1 ? 1 : (rs > kActSample ? kActSample : rs);
-  const auto at = [&](uint32_t i) { return keys[i]; };
-  const uint32_t lo = rs - half >= 1
-      ? block_select(at, kActSample, static_cast<uint32_t>(rs - half), hist, scratch) : 0u;
-  const uint32_t hi = rs + half <= kActSample
-      ? block_select(at, kActSample, static_cast<uint32_t>(rs + half), hist, scratch)
-      : 0xFFFFFFFFu;
+  const bool has_lo = rs - half >= 1, has_hi = rs + half <= kActSample;
+  const uint32_t k_lo = has_lo ? static_cast<uint32_t>(rs - half) : 1u;
+  const uint32_t k_hi = has_hi ? static_cast<uint32_t>(rs + half) : 1u;
+  const uint32_t incl = block_incl_scan(h0 + h1, scratch);
+  const uint32_t excl = incl - h0 - h1;
+  if (excl < k_lo && k_lo <= incl) bins[0] = b0 + (k_lo > excl + h0 ? 1u : 0u);
+  if (excl < k_hi && k_hi <= incl) bins[1] = b0 + (k_hi > excl + h0 ? 1u : 0u);
+  __syncthreads();
   if (threadIdx.x == 0) {
-    ws->lo = lo;
-    ws->hi = hi;
+    ws->lo = has_lo ? bins[0] << 20 : 0u;
+    ws->hi = has_hi ? (bins[1] << 20) | 0xFFFFFu : 0xFFFFFFFFu;
     ws->below = 0;
     ws->ncand = 0;
     ws->done = 0;
     ws->prefix = 0;
     ws->rank = rank;
+    ws->blocks_done = 0;
   }
 }
 
-__device__ __forceinline__ void bracket_one(uint32_t key, bool valid, uint32_t lo, uint32_t hi,
-                                            uint32_t& below, ActScaleWs* ws, int lane) {
-  below += (valid && key < lo) ? 1u : 0u;
-  const bool c = valid && key >= lo && key <= hi;
-  const uint32_t m = __ballot_sync(0xffffffffu, c);
-  if (m) {
-    const int leader = __ffs(m) - 1;
-    uint32_t base = 0;
-    if (lane == leader) base = atomicAdd(&ws->ncand, __popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    if (c) {
-      const uint32_t idx = base + __popc(m & ((1u << lane) - 1u));
-      if (idx < kActCandCap) ws->cand[idx] = key;
-    }
+constexpr int kActLocalCap = 2048;   // candidates one CTA buffers in shared memory
+
+__device__ __forceinline__ void bracket_one(uint32_t key, uint32_t lo, uint32_t hi,
+                                            uint32_t& below, uint32_t* buf, uint32_t* nbuf) {
+  below += key < lo ? 1u : 0u;
+  if (key >= lo && key <= hi) {   // rare: a few candidates per CTA
+    const uint32_t i = atomicAdd(nbuf, 1u);
+    if (i < kActLocalCap) buf[i] = key;
   }
 }
 
+// One pass: keys < lo are counted, keys in [lo, hi] are collected per CTA in
+// shared memory and appended to the workspace list with one reservation per
+// CTA.  A CTA that finds more than kActLocalCap candidates makes the list
+// count exceed its capacity, which sends the decision to the radix fallback.
 __global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x, int64_t nvec,
                                                    const float* __restrict__ tail, int ntail,
                                                    ActScaleWs* ws) {
   pdl_launch_dependents();
   pdl_wait_prior();
-  __shared__ uint32_t part[8];
+  __shared__ uint32_t buf[kActLocalCap];
+  __shared__ uint32_t nbuf, base, part[8];
+  if (threadIdx.x == 0) nbuf = 0;
+  __syncthreads();
   const uint32_t lo = ws->lo, hi = ws->hi;
-  const int lane = threadIdx.x & 31;
   uint32_t below = 0;
-  const int64_t warps = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  for (int64_t base = gw * 32; base < nvec; base += warps * 32) {   // warp-uniform trip count
-    const int64_t v = base + lane;
-    const bool valid = v < nvec;
-    const float4 q = valid ? __ldcs(x + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-    bracket_one(abs_key(q.x), valid, lo, hi, below, ws, lane);
-    bracket_one(abs_key(q.y), valid, lo, hi, below, ws, lane);
-    bracket_one(abs_key(q.z), valid, lo, hi, below, ws, lane);
-    bracket_one(abs_key(q.w), valid, lo, hi, below, ws, lane);
+  constexpr int kU = 4;   // float4 loads in flight per thread
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; v + (kU - 1) * step < nvec; v += kU * step) {
+    float4 q[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) q[u] = __ldcs(x + v + u * step);
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      bracket_one(abs_key(q[u].x), lo, hi, below, buf, &nbuf);
+      bracket_one(abs_key(q[u].y), lo, hi, below, buf, &nbuf);
+      bracket_one(abs_key(q[u].z), lo, hi, below, buf, &nbuf);
+      bracket_one(abs_key(q[u].w), lo, hi, below, buf, &nbuf);
+    }
   }
-  if (blockIdx.x == 0 && threadIdx.x < 32) {
-    const bool valid = lane < ntail;
-    bracket_one(valid ? abs_key(tail[lane]) : 0u, valid, lo, hi, below, ws, lane);
+  for (; v < nvec; v += step) {
+    const float4 q = __ldcs(x + v);
+    bracket_one(abs_key(q.x), lo, hi, below, buf, &nbuf);
+    bracket_one(abs_key(q.y), lo, hi, below, buf, &nbuf);
+    bracket_one(abs_key(q.z), lo, hi, below, buf, &nbuf);
+    bracket_one(abs_key(q.w), lo, hi, below, buf, &nbuf);
   }
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail)
+    bracket_one(abs_key(tail[threadIdx.x]), lo, hi, below, buf, &nbuf);
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
   if (lane == 0) part[threadIdx.x >> 5] = below;
   __syncthreads();
+  const uint32_t n = nbuf;
   if (threadIdx.x == 0) {
     uint32_t t = 0;
     for (int w = 0; w < (blockDim.x >> 5); ++w) t += part[w];
     if (t) atomicAdd(&ws->below, t);
+    // an overflowing CTA pushes the count past the capacity (fallback decides)
+    base = n == 0 ? 0u : atomicAdd(&ws->ncand, n <= kActLocalCap ? n : kActCandCap + 1u);
   }
+  __syncthreads();
+  if (n <= kActLocalCap)
+    for (uint32_t i = threadIdx.x; i < n; i += blockDim.x)
+      if (base + i < kActCandCap) ws->cand[base + i] = buf[i];
 }
+
+// Candidates staged in dynamic shared memory when they fit (kActSelSmemKeys),
+// else read from the workspace list in every radix pass.
+constexpr uint32_t kActSelSmemKeys = 48 * 1024;
 
 __global__ void __launch_bounds__(1024) act_bracket_select(ActScaleWs* ws, float* s_x) {
   pdl_launch_dependents();
   pdl_wait_prior();
+  extern __shared__ uint32_t ck[];
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t scratch[34];
   const uint32_t below = ws->below, n = ws->ncand, rank = ws->rank;
   if (!(below < rank && rank - below <= n && n <= kActCandCap)) return;   // radix decides
   const uint32_t* cand = ws->cand;
-  const uint32_t key =
-      block_select([&](uint32_t i) { return cand[i]; }, n, rank - below, hist, scratch);
+  // every candidate lies in [lo, max]: only the bits below the highest bit in
+  // which lo and the largest candidate differ can vary
+  __shared__ uint32_t wmax[32];
+  uint32_t key;
+  if (n <= kActSelSmemKeys) {
+    constexpr int kU = 8;
+    uint32_t kmax = 0;
+    uint32_t i = threadIdx.x;
+    for (; i + (kU - 1) * 1024 < n; i += kU * 1024) {
+      uint32_t v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) v[u] = cand[i + u * 1024];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        ck[i + u * 1024] = v[u];
+        kmax = v[u] > kmax ? v[u] : kmax;
+      }
+    }
+    for (; i < n; i += 1024) {
+      const uint32_t v = cand[i];
+      ck[i] = v;
+      kmax = v > kmax ? v : kmax;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = kmax;
+    __syncthreads();
+    kmax = wmax[threadIdx.x & 31];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    const uint32_t diff = (ws->lo ^ kmax) & 0x7FFFFFFFu;
+    const int top = diff ? 32 - __clz(diff) : 0;
+    key = block_select([&](uint32_t j) { return ck[j]; }, n, rank - below, hist, scratch, top,
+                       ws->lo);
+  } else {
+    const uint32_t diff = (ws->lo ^ ws->hi) & 0x7FFFFFFFu;
+    const int top = diff ? 32 - __clz(diff) : 0;
+    key = block_select([&](uint32_t j) { return cand[j]; }, n, rank - below, hist, scratch, top,
+                       ws->lo);
+  }
   if (threadIdx.x == 0) {
     const float t = __uint_as_float(key);
     *s_x = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
@@ -757,14 +864,21 @@ __global__ void __launch_bounds__(1024) act_bracket_select(ActScaleWs* ws, float
   }
 }
 
+// Radix pass p of the fallback: per-CTA shared histograms of bits [shift,
+// shift + bits) of the keys under the current prefix, merged into the
+// workspace; the last CTA to finish picks the bin holding the rank, narrows
+// the prefix and clears the histogram for the next pass (writing s_x after
+// the last pass).  Returns at once when the bracket path has decided.
 __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__ x, int64_t nvec,
                                                       const float* __restrict__ tail,
                                                       int ntail, ActScaleWs* ws, int shift,
-                                                      int bits, uint32_t hi_mask) {
+                                                      int bits, uint32_t hi_mask, float* s_x,
+                                                      int last_pass) {
   pdl_launch_dependents();
   pdl_wait_prior();
   if (ws->done) return;
   __shared__ uint32_t h[2048];
+  __shared__ uint32_t is_last;
   const uint32_t nb = 1u << bits;
   for (uint32_t i = threadIdx.x; i < nb; i += blockDim.x) h[i] = 0;
   __syncthreads();
@@ -789,22 +903,23 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
   __syncthreads();
   for (uint32_t i = threadIdx.x; i < nb; i += blockDim.x)
     if (h[i]) atomicAdd(&ws->hist[i], h[i]);
-}
-
-__global__ void act_scale_select(ActScaleWs* ws, int shift, int bits, float* s_x, int last) {
-  pdl_launch_dependents();
-  pdl_wait_prior();
-  if (threadIdx.x != 0 || ws->done) return;
-  const uint32_t nb = 1u << bits;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(&ws->blocks_done, 1u) == gridDim.x - 1u;
+  __syncthreads();
+  if (!is_last || threadIdx.x != 0) return;
+  __threadfence();
+  volatile uint32_t* vh = ws->hist;
   uint32_t below = 0, b = 0;
   for (b = 0; b < nb - 1u; ++b) {
-    if (below + ws->hist[b] >= ws->rank) break;
-    below += ws->hist[b];
+    if (below + vh[b] >= ws->rank) break;
+    below += vh[b];
   }
   ws->prefix |= b << shift;
   ws->rank -= below;
-  for (uint32_t i = 0; i < nb; ++i) ws->hist[i] = 0;
-  if (last) {
+  for (uint32_t i = 0; i < nb; ++i) vh[i] = 0;
+  ws->blocks_done = 0;
+  if (last_pass) {
     const float t = __uint_as_float(ws->prefix);
     *s_x = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
   }
@@ -1045,18 +1160,19 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
     const uint64_t bit = 1ull << (dev & 63);
-    const int sample_smem = kActSample * 4;
+    const int sel_smem = static_cast<int>(kActSelSmemKeys * 4);
     if (!(attr_set & bit)) {
       const cudaError_t e = cudaFuncSetAttribute(
-          act_sample, cudaFuncAttributeMaxDynamicSharedMemorySize, sample_smem);
+          act_bracket_select, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
       if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
       attr_set |= bit;
     }
-    SP24_TRY(launch_kernel(act_sample, dim3(1), dim3(1024), sample_smem, s, 1, X, count, rank,
-                           ws));
+    SP24_TRY(launch_kernel(act_sample_load, dim3(kActSampleCtas), dim3(1024), 0, s, 1, X,
+                           count, ws));
+    SP24_TRY(launch_kernel(act_sample_select, dim3(1), dim3(1024), 0, s, 1, count, rank, ws));
     SP24_TRY(launch_kernel(act_bracket, dim3(grid_for(nvec, 256)), dim3(256), 0, s, 1,
                            reinterpret_cast<const float4*>(X), nvec, X + nvec * 4, ntail, ws));
-    SP24_TRY(launch_kernel(act_bracket_select, dim3(1), dim3(1024), 0, s, 1, ws, s_x));
+    SP24_TRY(launch_kernel(act_bracket_select, dim3(1), dim3(1024), sel_smem, s, 1, ws, s_x));
   } else {
     SP24_TRY(launch_kernel(act_scale_init, dim3(1), dim3(256), 0, s, 1, ws, rank));
   }
@@ -1067,9 +1183,7 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
   for (int p = 0; p < 3; ++p) {
     SP24_TRY(launch_kernel(act_scale_hist, dim3(grid), dim3(256), 0, s, 1,
                            reinterpret_cast<const float4*>(X), nvec, X + nvec * 4, ntail, ws,
-                           shifts[p], bitsv[p], hi_mask));
-    SP24_TRY(launch_kernel(act_scale_select, dim3(1), dim3(32), 0, s, 1, ws, shifts[p],
-                           bitsv[p], s_x, static_cast<int>(p == 2)));
+                           shifts[p], bitsv[p], hi_mask, s_x, static_cast<int>(p == 2)));
     hi_mask |= ((1u << bitsv[p]) - 1u) << shifts[p];
   }
   return SP24_OK;
