@@ -235,7 +235,8 @@ struct CompressOut;
 enum { kValsNone = 0, kValsBF16 = 1, kValsINT8 = 2 };
 
 constexpr int kStreamStages = 5;
-constexpr int kStreamThreads = 1024;
+constexpr int kStreamThreads = 512;
+constexpr int kStreamRows = 128 / (kStreamThreads / 16);   // chunk rows per thread (4)
 constexpr int kWTile = 128 * 256;          // 128 rows x 128 bf16
 constexpr int kMTile = 128 * 16;           // 128 rows x 16 mask bytes
 constexpr int kNTile = 128 * 8;            // 128 float64 norms
@@ -271,7 +272,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
 
   const int tid = threadIdx.x;
   const uint32_t bb = tid & 15u;              // vector within a chunk row
-  const uint32_t m0 = tid >> 4;               // first chunk row (0..63)
+  const uint32_t m0 = tid >> 4;               // first chunk row (0..31)
   const int64_t kvec = a.k / 8;
   const int nmine = a.nchunks > static_cast<int>(blockIdx.x)
                         ? (a.nchunks - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
@@ -320,9 +321,9 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
       for (int e = 0; e < 8; ++e)
         nrm[e] = reinterpret_cast<const double*>(sb + kWTile + kMTile)[bb * 8 + e];
     }
-    // per-thread bases: chunk row m0 + 64 j is +16384 bytes of the W tile,
-    // +1024 bytes of the mask tile, of the metadata chunk (both layouts) and
-    // of the mask staging, and +64 j * kvec vectors in global memory
+    // per-thread bases: chunk row m0 + 32 j is +8192 bytes of the W tile,
+    // +512 bytes of the mask tile, of the metadata chunk (both layouts) and
+    // of the mask staging, and +32 j * kvec vectors in global memory
     const uint8_t* wrow = sb + m0 * 256 + bb * 16;
     const uint8_t* mrow = sb + kWTile + m0 * 16 + bb;
     const float* srow = reinterpret_cast<const float*>(sb + kWTile + kMTile + kNTile) + m0;
@@ -331,17 +332,17 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     const int64_t row0 = static_cast<int64_t>(rt) * 128 + m0;
     const int64_t vi0 = row0 * kvec + kv;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const bool ok = kv_ok && row0 + 64 * j < a.n;
-      const int64_t vi = vi0 + static_cast<int64_t>(64 * j) * kvec;
+    for (int j = 0; j < kStreamRows; ++j) {
+      const bool ok = kv_ok && row0 + 32 * j < a.n;
+      const int64_t vi = vi0 + static_cast<int64_t>(32 * j) * kvec;
       uint32_t meta_byte = 0x44u;             // padding: positions (0, 1)
       uint32_t keep = 0;
       if (ok) {
-        const uint4 q = *reinterpret_cast<const uint4*>(wrow + 16384 * j);
+        const uint4 q = *reinterpret_cast<const uint4*>(wrow + 8192 * j);
         uint32_t mbyte = 0xFFu;
         if (!kPrune || kMaskIn) {
           if (use_mask_tile) {
-            mbyte = mrow[1024 * j];
+            mbyte = mrow[512 * j];
           } else {
             mbyte = a.mask_direct[vi];
           }
@@ -375,7 +376,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
           if constexpr (kVals == kValsBF16) {
             __stcs(reinterpret_cast<uint2*>(a.vals) + vi, make_uint2(p0, p1));
           } else {
-            const float sc = srow[64 * j];
+            const float sc = srow[32 * j];
             const float xs[4] = {__uint_as_float(p0 << 16), __uint_as_float(p0 & 0xFFFF0000u),
                                  __uint_as_float(p1 << 16), __uint_as_float(p1 & 0xFFFF0000u)};
             uint32_t packed = 0;
@@ -389,8 +390,8 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
           }
         }
       }
-      if constexpr (kVals != kValsNone) mb[moff + 1024 * j] = meta_byte;
-      if (a.mask_out) ob[m0 * 16 + bb + 1024 * j] = static_cast<uint8_t>(keep);
+      if constexpr (kVals != kValsNone) mb[moff + 512 * j] = meta_byte;
+      if (a.mask_out) ob[m0 * 16 + bb + 512 * j] = static_cast<uint8_t>(keep);
     }
     __syncthreads();   // stage `st` fully read; chunk buffers complete
     if (tid == 0 && i + kStreamStages < nmine) {
@@ -926,8 +927,16 @@ __global__ void __launch_bounds__(256) act_scale_hist(const float4* __restrict__
 }
 
 // ----------------------------------------------------------- quantisation
-__device__ __forceinline__ uint32_t q8(float x, float s) {
-  int q = __float2int_rn(__fdiv_rn(x, s));
+// q = clamp(rint(x / s), -127, 127) with x / s the correctly rounded float32
+// quotient.  y = x * rcp(s) is within a few ulps of that quotient, so rint(y)
+// equals rint(x / s) unless a half-integer lies within that distance of y;
+// there (and for non-finite y) the quotient is formed exactly.
+__device__ __forceinline__ uint32_t q8(float x, float s, float rs) {
+  const float y = __fmul_rn(x, rs);
+  const float f = y - floorf(y);
+  float d = y;
+  if (!(fabsf(f - 0.5f) > 1e-5f * fabsf(y) + 1e-30f)) d = __fdiv_rn(x, s);
+  int q = __float2int_rn(d);
   q = q > 127 ? 127 : (q < -127 ? -127 : q);
   return static_cast<uint32_t>(q) & 0xFFu;
 }
@@ -938,14 +947,19 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float4* __restrict_
   pdl_launch_dependents();
   pdl_wait_prior();
   const float s = *s_ptr;
+  const float rs = __frcp_rn(s);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < nvec16;
        v += stride) {
+    float4 in[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) in[j] = __ldcs(x + 4 * v + j);
     uint32_t out[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 q = __ldcs(x + 4 * v + j);
-      out[j] = q8(q.x, s) | (q8(q.y, s) << 8) | (q8(q.z, s) << 16) | (q8(q.w, s) << 24);
+      const float4 q = in[j];
+      out[j] = q8(q.x, s, rs) | (q8(q.y, s, rs) << 8) | (q8(q.z, s, rs) << 16) |
+               (q8(q.w, s, rs) << 24);
     }
     xq[v] = make_uint4(out[0], out[1], out[2], out[3]);
   }
@@ -956,7 +970,7 @@ __global__ void quantize_tail(const float* __restrict__ x, int64_t start, int64_
   pdl_launch_dependents();
   pdl_wait_prior();
   const int64_t i = start + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i < count) xq[i] = static_cast<int8_t>(q8(x[i], *s_ptr));
+  if (i < count) xq[i] = static_cast<int8_t>(q8(x[i], *s_ptr, __frcp_rn(*s_ptr)));
 }
 
 

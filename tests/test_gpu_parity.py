@@ -262,6 +262,22 @@ def test_act_scale_large_coverages(kind, coverage):
     ok_status()
 
 
+@pytest.mark.parametrize("scale", [0.25, 0.0123457, 3.0])
+def test_quantize_half_integer_ties(scale):
+    # quotients at, and one float step either side of, every half-integer up
+    # to the clamp (rint: ties to even), plus values beyond the clamp
+    s = np.float32(scale)
+    halves = (np.arange(-140, 141, dtype=np.float64) + 0.5)
+    x = (halves * np.float64(s)).astype(np.float32)
+    near = np.concatenate([x, np.nextafter(x, np.float32(np.inf)),
+                           np.nextafter(x, np.float32(-np.inf)),
+                           np.array([1e30, -1e30, 0.0, -0.0], dtype=np.float32)])
+    xd = torch.from_numpy(near).cuda()
+    sd = torch.tensor([s, 0, 0, 0], dtype=torch.float32, device="cuda")[:1]
+    q = P.quantize(xd, sd)
+    assert np.array_equal(q.cpu().numpy(), O.quantize(near, s))
+
+
 def test_act_scale_and_quantize_int8_workload():
     w = I.int8_long_tail()
     xd = w.X.cuda()
