@@ -19,6 +19,7 @@ replica of the workload (weak scaling); time = max over ranks.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -225,6 +226,39 @@ class Runner:
         if self.wl.Xc is not None:
             t.append(self.wl.Xc)
         return t
+
+
+GEMM_SOURCES = ["gemm_sp.cu", "gemm_pair.cuh", "gemm_persistent.cuh", "gemm_epilogue.cuh",
+                "sp24_device.cuh", "sp24_host.h", "tma_host.h"]
+
+
+def gemm_src_hash() -> str:
+    """Hash of the GEMM kernel sources (the profiles record the one they were
+    captured with)."""
+    h = hashlib.sha256()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "structured_sparse_gemm_sp24_b200",
+                        "csrc")
+    for n in GEMM_SOURCES:
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def gemm_traffic(workload: str):
+    """DRAM bytes (read + write) of one GEMM launch on this workload from the
+    committed ncu summary table, or None when there is no row for it or the
+    kernel sources changed since it was captured."""
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
+                        "gemm_dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    cur = gemm_src_hash()
+    with open(path) as f:
+        for line in f:
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) == 4 and cells[0] == workload and cells[3] == cur:
+                return int(cells[2])
+    return None
 
 
 def time_steps(runner, steps, flush, stream, use_graph=True):
@@ -474,7 +508,7 @@ def main(argv=None):
     else:
         roof = {"bound": "hbm", "achieved": g_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": g_gbs / peaks["hbm_gbs"]}
-    roof["traffic"] = None
+    roof["traffic"] = gemm_traffic(wl.name)
     roof["peak_source"] = peaks["source"] + (" (2x dense bf16 burst)" if not wl.int8 else
                                              " (4x dense bf16 burst)")
     plan = B.sp24_gemm_plan(wl.M, wl.N, wl.K, B.SP24_INT8 if wl.int8 else B.SP24_BF16)
