@@ -468,9 +468,8 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
                        mb, me, my, my16, a);
 }
 
-// Which large-problem kernel to use: SP24_GEMM_IMPL = pair256 | pair240 |
-// pair224 | pair192 | pair128 | single (tuning override; default chooses by
-// problem size).
+// Which kernel to use: SP24_GEMM_IMPL = pair256 | pair240 | pair224 | pair192 |
+// pair128 | single | splitk (tuning override; default chooses by problem size).
 enum Impl : int { kSplitK = 0, kPair256 = 1, kPair128 = 2, kSingle = 3, kPair224 = 4,
                   kPair192 = 5, kPair240 = 6 };
 
@@ -483,7 +482,17 @@ int impl_override() {
   if (std::strcmp(e, "pair224") == 0) return kPair224;
   if (std::strcmp(e, "pair192") == 0) return kPair192;
   if (std::strcmp(e, "pair240") == 0) return kPair240;
+  if (std::strcmp(e, "splitk") == 0) return kSplitK;
   return -1;
+}
+
+// SP24_SPLITK = 1 | 2 | 4 | 8: K slices of the split-K kernel (tuning
+// override; 0 = choose by shape).
+int split_override() {
+  const char* e = std::getenv("SP24_SPLITK");
+  if (!e) return 0;
+  const int v = std::atoi(e);
+  return (v == 1 || v == 2 || v == 4 || v == 8) ? v : 0;
 }
 
 const char* impl_name(int impl) {
@@ -581,15 +590,16 @@ struct Plan {
 // The launch plan.  At least 128 tokens and enough 128 x 128 tiles for half
 // the SMs: a persistent kernel, the variant with the lowest estimated time (or
 // the SP24_GEMM_IMPL override).  Otherwise (few tokens or few tiles): the
-// split-K kernel, BN from the token count and K split until the CTAs cover
-// the SMs.
+// split-K kernel, BN from the token count and K split as far as all CTAs still
+// fit one wave (SP24_SPLITK overrides the split).
 sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
   const int sms = sm_count();
   const int64_t row_tiles = (n + 127) / 128;
-  if (m >= 128 && row_tiles * ((m + 127) / 128) >= sms / 2) {
+  const int forced = impl_override();
+  if (forced != kSplitK && m >= 128 && row_tiles * ((m + 127) / 128) >= sms / 2) {
     int pairs = 0;
     SP24_TRY(pair_capacity(&pairs));
-    int impl = impl_override();
+    int impl = forced;
     if (impl < 0) {
       impl = kSingle;   // pair tiles need both dimensions to fill them
       if (m >= 256 && n >= 256) {
@@ -624,8 +634,15 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
   }
   const int bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
   const int64_t base = row_tiles * ((m + bn - 1) / bn);
+  // one CTA per SM fits (the rings take most of shared memory), so the K
+  // split stops where the CTAs would exceed one wave: measured on B200 for
+  // M = 16..256 decode shapes, a second wave costs more than the longer K
+  // loop of a smaller split (e.g. M = 16, 11008 x 4096: split 1 on 86 SMs
+  // 20.5 us, split 4 on 344 CTAs 29 us)
   int split = 1;
-  while (split < 8 && base * split < 2 * sms && kblocks >= 2 * split) split *= 2;
+  while (split < 8 && base * split * 2 <= sms && kblocks >= 4 * split) split *= 2;
+  const int so = split_override();
+  if (so > 0 && so <= kblocks) split = so;
   p->impl = kSplitK;
   p->bn = bn;
   p->split = split;

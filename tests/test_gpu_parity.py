@@ -496,6 +496,27 @@ def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
     ok_status()
 
 
+@pytest.mark.parametrize("split", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("mnk", [(16, 392, 1024), (40, 264, 2048 + 128), (128, 136, 1536)])
+def test_gemm_splitk_forced(split, mnk, monkeypatch):
+    # every K split of the split-K kernel (the plan picks few of them)
+    monkeypatch.setenv("SP24_GEMM_IMPL", "splitk")
+    monkeypatch.setenv("SP24_SPLITK", split)
+    m, n, k = mnk
+    plan = B.sp24_gemm_plan(m, n, k, B.SP24_BF16)
+    assert plan["kernel"] == "splitk" and plan["split_k"] == int(split)
+    W = I.normal_bf16((n, k), 1.0, seed=61)
+    X = I.normal_bf16((m, k), 1.0, seed=62)
+    _, _, _, y = _bf16_pipeline(W, X)
+    assert_bf16_close(y, *_bf16_ref(W, X))
+    acc, s_x, s_w = _int8_ref(I.long_tail_bf16((n, k), 0.02, seed=63, tail_seed=64),
+                              I.normal_f32((m, k), 1.0, seed=65))
+    yi, _, _ = _int8_pipeline(I.long_tail_bf16((n, k), 0.02, seed=63, tail_seed=64),
+                              I.normal_f32((m, k), 1.0, seed=65), B.SP24_OUT_INT32)
+    assert np.array_equal(yi.cpu().numpy(), acc)
+    ok_status()
+
+
 # ------------------------------------------------------------ launch plans
 def test_gemm_plan_families(monkeypatch):
     monkeypatch.delenv("SP24_GEMM_IMPL", raising=False)
