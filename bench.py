@@ -228,36 +228,45 @@ class Runner:
         return t
 
 
-GEMM_SOURCES = ["gemm_sp.cu", "gemm_pair.cuh", "gemm_persistent.cuh", "gemm_epilogue.cuh",
-                "sp24_device.cuh", "sp24_host.h", "tma_host.h"]
+COMMON_SOURCES = ["sp24_device.cuh", "sp24_host.h", "tma_host.h"]
+FAMILY_SOURCES = {   # the files that define each GEMM kernel family and its launch
+    "pair": ["gemm_pair.cuh", "gemm_epilogue.cuh"] + COMMON_SOURCES,
+    "single": ["gemm_persistent.cuh", "gemm_epilogue.cuh"] + COMMON_SOURCES,
+    "splitk": ["gemm_splitk.cuh"] + COMMON_SOURCES,
+}
 
 
-def gemm_src_hash() -> str:
-    """Hash of the GEMM kernel sources (the profiles record the one they were
-    captured with)."""
+def family_of(plan_kernel: str) -> str:
+    return "pair" if plan_kernel.startswith("pair") else plan_kernel
+
+
+def gemm_src_hash(family: str) -> str:
+    """Hash of the sources of one GEMM kernel family (the profiles record the
+    one they were captured with)."""
     h = hashlib.sha256()
     csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "structured_sparse_gemm_sp24_b200",
                         "csrc")
-    for n in GEMM_SOURCES:
+    for n in FAMILY_SOURCES[family]:
         with open(os.path.join(csrc, n), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def gemm_traffic(workload: str):
+def gemm_traffic(workload: str, plan_kernel: str):
     """DRAM bytes (read + write) of one GEMM launch on this workload from the
-    committed ncu summary table, or None when there is no row for it or the
-    kernel sources changed since it was captured."""
+    committed ncu summary table, or None when there is no row for it, the plan
+    now picks another kernel, or that kernel's sources changed since."""
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles",
                         "gemm_dram_traffic.md")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or family_of(plan_kernel) not in FAMILY_SOURCES:
         return None
-    cur = gemm_src_hash()
+    cur = gemm_src_hash(family_of(plan_kernel))
     with open(path) as f:
         for line in f:
             cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) == 4 and cells[0] == workload and cells[3] == cur:
-                return int(cells[2])
+            if (len(cells) == 5 and cells[0] == workload and cells[1] == plan_kernel
+                    and cells[4] == cur):
+                return int(cells[3])
     return None
 
 
@@ -508,10 +517,10 @@ def main(argv=None):
     else:
         roof = {"bound": "hbm", "achieved": g_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": g_gbs / peaks["hbm_gbs"]}
-    roof["traffic"] = gemm_traffic(wl.name)
     roof["peak_source"] = peaks["source"] + (" (2x dense bf16 burst)" if not wl.int8 else
                                              " (4x dense bf16 burst)")
     plan = B.sp24_gemm_plan(wl.M, wl.N, wl.K, B.SP24_INT8 if wl.int8 else B.SP24_BF16)
+    roof["traffic"] = gemm_traffic(wl.name, plan["kernel"])
     roof["kernel"] = "sp24 gemm " + plan["kernel"]
     roof["plan"] = plan
     c_gbs = runner.compress_bytes() / (comp_ms * 1e-3) / 1e9

@@ -229,4 +229,127 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   if (warp == 2) tmem_dealloc_pair(tmem_base, C::kTmemCols);
 }
 
+// ------------------------------------------------------------ host launch
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
+sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x, int pairs,
+                        cudaStream_t s) {
+  using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
+  auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC>;
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    attr_set |= bit;
+  }
+  const int el = kDtype == SP24_BF16 ? 2 : 1;
+  const CUtensorMapDataType dt =
+      kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  // B: each CTA loads BN/2 token rows
+  CUtensorMap mb;
+  SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(g.k), static_cast<uint64_t>(g.m),
+                    static_cast<uint32_t>(128 / el), static_cast<uint32_t>(C::kHalfN)));
+  // E: metadata chunks as rows of 256 bytes (8 rows per 2048-byte chunk)
+  const int64_t kchunks = (g.k + 127) / 128;
+  const int64_t rt128 = (g.n + 127) / 128;
+  CUtensorMap me;
+  SP24_TRY(make_map(&me, g.meta, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, 32,
+                    static_cast<uint64_t>(rt128 * kchunks * 8), 32,
+                    static_cast<uint32_t>(8 * C::kMetaChunks), CU_TENSOR_MAP_SWIZZLE_NONE));
+  const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                  : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int y_box = epi_box(g.n);
+  const CUtensorMapSwizzle yswz =
+      epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUtensorMap my, my16;
+  SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk, yswz));
+  // tiles of 16 (mod 32) tokens store their last chunk with 16-token boxes
+  if (BN % kEpiChunk != 0) {
+    SP24_TRY(make_map(&my16, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                      static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), 16, yswz));
+  } else {
+    my16 = my;
+  }
+  PersistArgs a;
+  a.meta = g.meta;
+  a.s_x = g.s_x;
+  a.s_w = g.s_w;
+  a.s_y = g.s_y;
+  a.m = g.m;
+  a.n = g.n;
+  a.k = g.k;
+  a.kblocks = g.kblocks;
+  a.row_tiles = static_cast<int>((g.n + 255) / 256);
+  a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
+  const int64_t row_tile_bytes = 256 * (g.k / 2) * el;
+  int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
+  a.group_rows = static_cast<int>(gr);
+  a.y_box = y_box;
+  const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
+  if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
+  if (pairs < 1 || pairs > ntiles) return SP24_ERR_ARG;   // the plan sizes the grid
+  return launch_kernel(kern, dim3(2 * pairs), dim3(64 + kEpiThreads), C::kSmemBytes, s, 2, ma,
+                       mb, me, my, my16, a);
+}
+
+// CTA pairs (clusters of 2) that can be resident at once.  A cluster lives in
+// one GPC, so a GPC with an odd number of SMs leaves one out and the count can
+// be below SMs / 2; the persistent pair kernels launch exactly this many pairs
+// so that no pair waits for another to finish.  Every pair variant holds one
+// CTA per SM, so one query (cached per device) serves them all.
+inline sp24_status pair_capacity(int* out) {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  if (cache[dev & 63] > 0) {
+    *out = cache[dev & 63];
+    return SP24_OK;
+  }
+  using C = PairCfg<SP24_BF16, 256, 4, SP24_OUT_BF16, 1>;
+  auto kern = gemm_sp_pair<SP24_BF16, 256, 4, SP24_OUT_BF16, 1>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+  cfg.blockDim = dim3(64 + kEpiThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters", e);
+  if (n < 1) return SP24_ERR_UNSUPPORTED;
+  cache[dev & 63] = n;
+  *out = n;
+  return SP24_OK;
+}
+
+// CTA-pair kernel for every output kind; ST = ring stages (ST32 with int32
+// output, whose staging is twice the size).
+template <int kDtype, int BN, int ST, int ST32, int ACC>
+sp24_status launch_pair_out(const CUtensorMap& ma, const GemmArgs& a, const void* x, int pairs,
+                            cudaStream_t s) {
+  if constexpr (kDtype == SP24_BF16) {
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, pairs, s);
+  } else {
+    if (a.out_kind == SP24_OUT_INT32)
+      return launch_pair<kDtype, BN, ST32, SP24_OUT_INT32, ACC>(ma, a, x, pairs, s);
+    if (a.out_kind == SP24_OUT_INT8)
+      return launch_pair<kDtype, BN, ST, SP24_OUT_INT8, ACC>(ma, a, x, pairs, s);
+    return launch_pair<kDtype, BN, ST, SP24_OUT_BF16, ACC>(ma, a, x, pairs, s);
+  }
+}
+
 }  // namespace sp24

@@ -232,4 +232,53 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
   if (warp == 2) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ------------------------------------------------------------ host launch
+template <int kDtype, int BN, int STAGES, int OUTK>
+sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g,
+                              cudaStream_t s) {
+  using C = PersistCfg<kDtype, BN, STAGES, OUTK>;
+  auto kern = gemm_sp_persistent<kDtype, BN, STAGES, OUTK>;
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(attr_set & bit)) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+    attr_set |= bit;
+  }
+  const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                  : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                          : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const int y_box = epi_box(g.n);
+  CUtensorMap my;
+  SP24_TRY(make_map(&my, g.y, ydt, C::kOutBytes, static_cast<uint64_t>(g.n),
+                    static_cast<uint64_t>(g.m), static_cast<uint32_t>(y_box), kEpiChunk,
+                    epi_vec<OUTK>(g.n) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE));
+  PersistArgs a;
+  a.meta = g.meta;
+  a.s_x = g.s_x;
+  a.s_w = g.s_w;
+  a.s_y = g.s_y;
+  a.m = g.m;
+  a.n = g.n;
+  a.k = g.k;
+  a.kblocks = g.kblocks;
+  a.row_tiles = static_cast<int>((g.n + 127) / 128);
+  a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
+  // raster group: as many weight row tiles as fit ~24 MB of compressed weights
+  const int64_t row_tile_bytes = 128 * (g.k / 2) * (kDtype == SP24_BF16 ? 2 : 1);
+  int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
+  a.group_rows = static_cast<int>(gr);
+  a.y_box = y_box;
+  const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
+  if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(ntiles < sm_count() ? ntiles : sm_count());
+  return launch_kernel(kern, dim3(grid), dim3(64 + kEpiThreads), C::kSmemBytes, s, 1, ma, mb, my,
+                       a);
+}
+
+
 }  // namespace sp24

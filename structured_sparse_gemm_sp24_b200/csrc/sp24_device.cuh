@@ -190,6 +190,15 @@ __device__ __forceinline__ void tc_mma_sp_i8(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
+// Instruction descriptor of tcgen05.mma.sp (M = 128, K-major A and B).
+template <int kDtype, int BN>
+__device__ __forceinline__ uint32_t make_idesc(uint32_t id2) {
+  const uint32_t c_fmt = kDtype == SP24_BF16 ? 1u : 2u;  // F32 : S32
+  const uint32_t ab_fmt = 1u;                             // BF16 : signed int8
+  return (id2 & 3u) | (1u << 2) | (c_fmt << 4) | (ab_fmt << 7) | (ab_fmt << 10) |
+         (static_cast<uint32_t>(BN >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 // Each thread of the warp reads 16 consecutive 32-bit columns of its own lane
 // (warp w of the CTA reaches lanes 32*(w%4) .. 32*(w%4)+31).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
