@@ -149,10 +149,11 @@ class Runner:
     def launches_per_step(self) -> int:
         if self.wl.int8:
             return 1 + 1 + 1 + 7 + 1 + 1     # prune, wscale, compress, act_scale, quantize, gemm
-        if self.wanda and self.wl.progressive:
-            return 2 + 1 + 1                 # colnorm+prune(3:4), prune_compress, gemm
         if self.wanda:
-            return 2 + 1 + 1
+            # the library forms the column norms inside the prune kernel when
+            # row tiles x calibration rows is small, else launches colnorm first
+            fused = ((self.N + 127) // 128) * self.wl.Xc.shape[0] <= 8192
+            return (1 if fused else 2) + 1 + 1   # [colnorm +] prune, prune_compress, gemm
         return 1 + 1                         # prune_compress, gemm
 
     def step(self, ev=None):
@@ -321,6 +322,36 @@ def time_steps(runner, steps, flush, stream, use_graph=True):
     return tot, prune, comp, gemm
 
 
+def count_step_kernels(runner):
+    """Kernels in one step, counted as the kernel nodes of a CUDA graph captured
+    from it (every kernel in the step is a library kernel); None if the graph
+    cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as cudart
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g):
+            runner.step()
+        raw = g.raw_cuda_graph()
+        h = raw if isinstance(raw, cudart.cudaGraph_t) else cudart.cudaGraph_t(init_value=int(raw))
+        err, _, n = cudart.cudaGraphGetNodes(h, 0)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = cudart.cudaGraphGetNodes(h, n)
+        if err != cudart.cudaError_t.cudaSuccess:
+            return None
+        kern = cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        count = 0
+        for nd in nodes[:n]:
+            e2, t = cudart.cudaGraphNodeGetType(nd)
+            if e2 == cudart.cudaError_t.cudaSuccess and t == kern:
+                count += 1
+        g.reset()
+        return count
+    except Exception as exc:   # no cuda-python or no raw graph access
+        print(f"bench: could not count graph kernel nodes ({exc})", file=sys.stderr)
+        return None
+
+
 def time_e2e(runner, steps, device):
     """Same step through host buffers: pinned H2D copies of the step's inputs and
     a D2H copy of Y inside the timed region."""
@@ -469,6 +500,11 @@ def main(argv=None):
             dist.barrier()
         torch.cuda.synchronize()
 
+    counted = count_step_kernels(runner)
+    step_kernels = counted if counted is not None else runner.launches_per_step()
+    if counted is not None and counted != runner.launches_per_step():
+        print(f"bench: step graph holds {counted} kernels, expected "
+              f"{runner.launches_per_step()}", file=sys.stderr)
     barrier()
     with ClockSampler(local) as clk:
         tot, prune, comp, gemm = time_steps(runner, args.steps, flush, stream,
@@ -543,7 +579,7 @@ def main(argv=None):
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": runner.launches_per_step() * args.steps,
+        "gpu_launches": step_kernels * args.steps,
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

@@ -243,6 +243,8 @@ constexpr int kNTile = 128 * 8;            // 128 float64 norms
 constexpr int kSTile = 128 * 4;            // 128 float32 row scales
 constexpr int kStreamStage = kWTile + kMTile + kNTile + kSTile;   // multiple of 128
 constexpr int kStreamSmem = kStreamStages * kStreamStage + 4 * 2048 + 256 + 1024;
+constexpr int kXcTile = 128 * 256;   // fused Wanda norms: 128 tokens x 128 columns of Xc
+constexpr int kStreamSmemFused = kStreamSmem + kXcTile;
 
 struct StreamArgs {
   int64_t n, k;
@@ -254,6 +256,12 @@ struct StreamArgs {
   uint8_t* mask_out;           // NULL: not written
   void* vals;
   uint8_t* meta;
+  // Wanda with the column norms computed in the kernel (xc != NULL): each CTA
+  // forms the norms of its chunk's 128 columns from Xc [mc][k]; CTAs of row
+  // tile 0 also store them to norms_out
+  const uint16_t* xc;
+  int64_t mc;
+  double* norms_out;
 };
 
 template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
@@ -278,7 +286,9 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                         ? (a.nchunks - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x
                         : 0;
   const bool use_mask_tile = a.mask_tma != 0;
-  const uint32_t stage_tx = kWTile + (use_mask_tile ? kMTile : 0) + (kWanda ? kNTile : 0) +
+  const bool fused_norms = kWanda && a.xc != nullptr;
+  const uint32_t stage_tx = kWTile + (use_mask_tile ? kMTile : 0) +
+                            ((kWanda && !fused_norms) ? kNTile : 0) +
                             (kVals == kValsINT8 ? kSTile : 0);
 
   if (tid == 0) {
@@ -295,7 +305,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     mbar_arrive_expect_tx(&full[st], stage_tx);
     tma_load_2d(sb, &tm_w, &full[st], kb * 128, rt * 128);
     if (use_mask_tile) tma_load_2d(sb + kWTile, &tm_mask, &full[st], kb * 16, rt * 128);
-    if constexpr (kWanda) tma_load_1d(sb + kWTile + kMTile, &tm_norm, &full[st], kb * 128);
+    if (kWanda && !fused_norms) tma_load_1d(sb + kWTile + kMTile, &tm_norm, &full[st], kb * 128);
     if constexpr (kVals == kValsINT8)
       tma_load_1d(sb + kWTile + kMTile + kNTile, &tm_sw, &full[st], rt * 128);
   };
@@ -317,6 +327,50 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     uint8_t* ob = mout_buf + (i & 1) * 2048;
     double nrm[8];
     if constexpr (kWanda) {
+      if (fused_norms) {
+        // column norms of this chunk, in the stage's norm slot (TMA does not
+        // write it in this mode): Xc is staged 128 tokens at a time with
+        // every 16-byte load in flight; threads 0..127 then add the squares
+        // of their column in token order (float64, one rounding per product
+        // and per addition), then sqrt
+        // 256 bytes past the stage barriers (16-byte aligned), in the kXcTile
+        // bytes a fused launch adds to the dynamic shared memory
+        uint16_t(*xt)[128] = reinterpret_cast<uint16_t(*)[128]>(full + 32);
+        const int64_t col0 = static_cast<int64_t>(kb) * 128;
+        const int cvalid = static_cast<int>(a.k - col0 < 128 ? a.k - col0 : 128);   // % 8 == 0
+        double acc = 0.0;
+        for (int64_t t0 = 0; t0 < a.mc; t0 += 128) {
+          const int rows = static_cast<int>(a.mc - t0 < 128 ? a.mc - t0 : 128);
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {   // 128 rows x 16 pieces of 8 columns
+            const int q = tid + u * kStreamThreads;
+            const int r = q >> 4, c8 = (q & 15) * 8;
+            if (r < rows && c8 < cvalid)
+              v[u] = __ldg(reinterpret_cast<const uint4*>(a.xc + (t0 + r) * a.k + col0 + c8));
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int q = tid + u * kStreamThreads;
+            const int r = q >> 4, c8 = (q & 15) * 8;
+            if (r < rows && c8 < cvalid) *reinterpret_cast<uint4*>(&xt[r][c8]) = v[u];
+          }
+          __syncthreads();
+          if (tid < cvalid) {
+            for (int r = 0; r < rows; ++r) {
+              const double x = bf16_to_double(xt[r][tid]);
+              acc = __dadd_rn(acc, __dmul_rn(x, x));
+            }
+          }
+          __syncthreads();
+        }
+        if (tid < 128) {
+          const double nv = __dsqrt_rn(acc);
+          reinterpret_cast<double*>(const_cast<uint8_t*>(sb) + kWTile + kMTile)[tid] = nv;
+          if (rt == 0 && tid < cvalid) a.norms_out[col0 + tid] = nv;
+        }
+        __syncthreads();
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e)
         nrm[e] = reinterpret_cast<const double*>(sb + kWTile + kMTile)[bb * 8 + e];
@@ -1023,7 +1077,8 @@ static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double*
 template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
 static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* mask_out,
                                  const double* norms, const float* s_w, int64_t n, int64_t k,
-                                 int n_keep, void* vals, void* meta, cudaStream_t s) {
+                                 int n_keep, void* vals, void* meta, cudaStream_t s,
+                                 const void* xc, int64_t mc) {
   auto kern = stream_kernel<kPrune, kWanda, kVals, kMaskIn>;
   static uint64_t attr_set = 0;   // one bit per device
   int dev = 0;
@@ -1031,7 +1086,8 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
   if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   const uint64_t bit = 1ull << (dev & 63);
   if (!(attr_set & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kWanda ? kStreamSmemFused : kStreamSmem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
     attr_set |= bit;
   }
@@ -1048,7 +1104,7 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
     SP24_TRY(make_map(&tm, mask, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, static_cast<uint64_t>(k / 8),
                       static_cast<uint64_t>(n), 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE));
   tn = tw;
-  if (kWanda)
+  if (kWanda && xc == nullptr)
     SP24_TRY(make_map_1d(&tn, norms, CU_TENSOR_MAP_DATA_TYPE_FLOAT64, static_cast<uint64_t>(k),
                          128));
   ts = tw;
@@ -1066,9 +1122,12 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
   a.mask_out = mask_out;
   a.vals = vals;
   a.meta = static_cast<uint8_t*>(meta);
+  a.xc = static_cast<const uint16_t*>(xc);
+  a.mc = mc;
+  a.norms_out = const_cast<double*>(norms);
   const int grid = static_cast<int>(nchunks < sm_count() ? nchunks : sm_count());
-  return launch_kernel(kern, dim3(grid), dim3(kStreamThreads), kStreamSmem, s, 1, tw, tm, tn, ts,
-                       a);
+  const int smem = (kWanda && xc != nullptr) ? kStreamSmemFused : kStreamSmem;
+  return launch_kernel(kern, dim3(grid), dim3(kStreamThreads), smem, s, 1, tw, tm, tn, ts, a);
 }
 
 // For the pruning variants `mask` is mask_in (optional); a separate
@@ -1076,12 +1135,29 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
 template <bool kPrune, bool kWanda, int kVals>
 static sp24_status launch_stream(const void* w, const uint8_t* mask, uint8_t* mask_out,
                                  const double* norms, const float* s_w, int64_t n, int64_t k,
-                                 int n_keep, void* vals, void* meta, cudaStream_t s) {
+                                 int n_keep, void* vals, void* meta, cudaStream_t s,
+                                 const void* xc = nullptr, int64_t mc = 0) {
   if (kPrune && mask == nullptr)
     return launch_stream_t<kPrune, kWanda, kVals, false>(w, mask, mask_out, norms, s_w, n, k,
-                                                         n_keep, vals, meta, s);
+                                                         n_keep, vals, meta, s, xc, mc);
   return launch_stream_t<kPrune, kWanda, kVals, true>(w, mask, mask_out, norms, s_w, n, k, n_keep,
-                                                      vals, meta, s);
+                                                      vals, meta, s, xc, mc);
+}
+
+// Wanda pruning: the column norms go to `norms` either from a separate
+// colnorm launch or, when recomputing them per row tile is cheap (row tiles x
+// calibration rows small), inside the prune kernel itself (one launch fewer).
+constexpr int64_t kFusedNormWork = 8192;   // max row tiles x Mc for the fused path
+
+static sp24_status launch_wanda_prune(const void* W, const uint8_t* mask_in, uint8_t* mask_out,
+                                      double* norms, int64_t N, int64_t K, const void* Xc,
+                                      int64_t Mc, int n_keep, cudaStream_t s) {
+  if (((N + 127) / 128) * Mc <= kFusedNormWork)
+    return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K, n_keep,
+                                                nullptr, nullptr, s, Xc, Mc);
+  SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
+  return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K, n_keep,
+                                              nullptr, nullptr, s);
 }
 
 }  // namespace sp24
@@ -1112,10 +1188,8 @@ sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc, int6
   SP24_TRY(check_device());
   cudaStream_t s = as_stream(stream);
   if (mode == SP24_WANDA) {
-    double* norms = static_cast<double*>(workspace);
-    SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
-    return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K,
-                                                n_keep, nullptr, nullptr, s);
+    return launch_wanda_prune(W, mask_in, mask_out, static_cast<double*>(workspace), N, K, Xc,
+                              Mc, n_keep, s);
   }
   return launch_stream<true, false, kValsNone>(W, mask_in, mask_out, nullptr, nullptr, N, K,
                                                n_keep, nullptr, nullptr, s);
@@ -1134,10 +1208,8 @@ sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const 
   SP24_TRY(check_device());
   double* norms = nullptr;
   SP24_TRY(noalloc_norms(&norms));
-  cudaStream_t s = as_stream(stream);
-  SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
-  return launch_stream<true, true, kValsNone>(W, mask_in, mask_out, norms, nullptr, N, K, n_keep,
-                                              nullptr, nullptr, s);
+  return launch_wanda_prune(W, mask_in, mask_out, norms, N, K, Xc, Mc, n_keep,
+                            as_stream(stream));
 }
 
 sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K,

@@ -108,6 +108,23 @@ def test_prune_wanda_bert(n_keep):
     assert np.array_equal(keep_of(mask, w.K), ref)
 
 
+@pytest.mark.parametrize("n,k,mc", [(130, 264, 37), (3072, 768, 128), (9000, 256, 128)])
+def test_prune_wanda_norm_paths(n, k, mc):
+    # small row-tiles x Mc: norms formed inside the prune kernel; large (the
+    # last case: 71 row tiles x 128): separate column-norm kernel.  Either way
+    # the mask matches and the workspace holds the norms afterwards.
+    W = I.normal_bf16((n, k), 0.02, seed=91)
+    Xc = I.normal_bf16((mc, k), 1.0, seed=92)
+    out = torch.empty((n, k // 8), dtype=torch.uint8, device="cuda")
+    ws = torch.full((B.sp24_prune_workspace_bytes(k, B.SP24_WANDA),), 0xAB, dtype=torch.uint8,
+                    device="cuda")
+    B.sp24_prune(W.cuda(), Xc.cuda(), B.SP24_WANDA, 2, None, out, ws)
+    ok_status()
+    assert np.array_equal(keep_of(out, k), O.prune(f64(W), O.WANDA, 2, xc=f64(Xc)))
+    norms = ws[: 8 * k].view(torch.float64).cpu().numpy()
+    assert np.array_equal(norms, O.column_norms(f64(Xc)))
+
+
 def test_progressive_bert():
     w = I.bert_fc1()
     Wd, Xc = w.W.cuda(), w.Xc.cuda()
