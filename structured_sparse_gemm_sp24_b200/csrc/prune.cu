@@ -234,7 +234,7 @@ struct CompressOut;
 // memory and written with 16-byte stores.
 enum { kValsNone = 0, kValsBF16 = 1, kValsINT8 = 2 };
 
-constexpr int kStreamStages = 5;
+constexpr int kStreamStages = 2;   // two CTAs per SM each keep two chunks in flight
 constexpr int kStreamThreads = 512;
 constexpr int kStreamRows = 128 / (kStreamThreads / 16);   // chunk rows per thread (4)
 constexpr int kWTile = 128 * 256;          // 128 rows x 128 bf16
@@ -1125,8 +1125,15 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
   a.xc = static_cast<const uint16_t*>(xc);
   a.mc = mc;
   a.norms_out = const_cast<double*>(norms);
-  const int grid = static_cast<int>(nchunks < sm_count() ? nchunks : sm_count());
   const int smem = (kWanda && xc != nullptr) ? kStreamSmemFused : kStreamSmem;
+  // as many persistent CTAs as fit (two per SM: one's barrier and TMA waits
+  // overlap the other's work)
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStreamThreads, smem);
+  if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveBlocksPerMultiprocessor", e);
+  if (per_sm < 1) return SP24_ERR_UNSUPPORTED;
+  const int64_t ctas = static_cast<int64_t>(sm_count()) * per_sm;
+  const int grid = static_cast<int>(nchunks < ctas ? nchunks : ctas);
   return launch_kernel(kern, dim3(grid), dim3(kStreamThreads), smem, s, 1, tw, tm, tn, ts, a);
 }
 
