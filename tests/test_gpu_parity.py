@@ -390,6 +390,26 @@ def test_gemm_bf16_square(n):
     assert_bf16_close(y[torch.from_numpy(rows).cuda()], yr, ar)
 
 
+@pytest.mark.parametrize("n", [2048, 8192, 16384])
+def test_gemm_bf16_square_sampled_large(n):
+    # up to the largest configured size: the whole pipeline runs on the GPU;
+    # sampled weight rows (pruning is row-independent) are pruned by the
+    # oracle, their masks compared bit for bit, and the outputs of sampled
+    # tokens x those channels checked against the float64 product
+    w = I.square(n)
+    mask, _, _, y = _bf16_pipeline(w.W, w.X)
+    ok_status()
+    cols = np.unique(np.r_[0:24, n - 24:n, 777:n:1999])
+    rows = np.unique(np.r_[0:16, n - 16:n, 100:n:2011])
+    Wc = w.W[torch.from_numpy(cols)]
+    keep = O.prune(f64(Wc), O.MAGNITUDE, 2)
+    assert np.array_equal(keep_of(mask[torch.from_numpy(cols).cuda()], n), keep)
+    vals, meta = O.compress(f64(Wc), keep)
+    yr, ar = O.gemm(f64(w.X[torch.from_numpy(rows)]), vals, meta, n)
+    got = y[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()]
+    assert_bf16_close(got, yr, ar)
+
+
 def test_gemm_bf16_deterministic_split():
     w = I.llm_proj(4096, 11008, 16)      # split-K over a cluster
     _, vals, meta, y1 = _bf16_pipeline(w.W, w.X)
