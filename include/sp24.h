@@ -135,8 +135,11 @@ sp24_status sp24_wscale(const void* W, const uint8_t* mask, int64_t N, int64_t K
 
 /* Per-tensor activation scale: t = the r-th smallest |X[i]| over all `count`
  * float32 values, r = max(1, ceil(coverage * count)) in IEEE double;
- * *s_x = t / 127.0f (float32), or 1 when t == 0.  Exact (radix selection on
- * the float32 bit patterns).
+ * *s_x = t / 127.0f (float32), or 1 when t == 0.  Exact order statistic of the
+ * float32 bit patterns: a bracket from a stratified sample is checked exactly
+ * against the counts of one pass over X and the answer selected among the
+ * values inside it; when the check fails (central coverages, heavy ties)
+ * three exact radix passes decide.
  *   X: float32 [count].  s_x: one float32 (device).
  *   workspace: sp24_act_scale_workspace_bytes() bytes.
  * Rules: count >= 1, 0 < coverage <= 1. */
@@ -259,6 +262,16 @@ sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const 
                                      uint8_t* mask_out, void* stream);
 
 /* --------------------------------------------------------------- status */
+
+/* Self-test of the failure path (the pages have no counterpart): launches one
+ * thread that waits, with the same bounded mbarrier wait every kernel of the
+ * library uses but a limit of limit_ns nanoseconds (1 .. 1e9), on a barrier
+ * nothing arrives at.  The wait gives up, records SP24_ERR_TIMEOUT in the
+ * device status word and the kernel returns normally: nothing traps or
+ * hangs, and the context stays usable.  The next sp24_device_status() on the
+ * stream reports (and clears) SP24_ERR_TIMEOUT.
+ * Errors: SP24_ERR_ARG for a limit out of range. */
+sp24_status sp24_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
  * current device (SP24_OK, SP24_ERR_PATTERN or SP24_ERR_TIMEOUT), or

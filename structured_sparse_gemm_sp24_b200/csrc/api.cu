@@ -1,4 +1,5 @@
 // libsp24: size queries, status word, error strings, device checks.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -9,8 +10,8 @@ namespace sp24 {
 
 namespace {
 constexpr int kMaxDevices = 64;
-int g_dev_ok[kMaxDevices];   // 0 unknown, 1 sm_100, 2 other
-int g_dev_sms[kMaxDevices];
+std::atomic<int> g_dev_ok[kMaxDevices];   // 0 unknown, 1 sm_100, 2 other
+std::atomic<int> g_dev_sms[kMaxDevices];
 std::mutex g_dev_mu;
 }  // namespace
 
@@ -29,23 +30,39 @@ sp24_status check_device() {
   const cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kMaxDevices) return SP24_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (g_dev_ok[dev] == 0) {
-    int major = 0, sms = 0;
-    cudaError_t a = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    if (a == cudaSuccess) a = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (a != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", a);
-    g_dev_ok[dev] = (major == 10) ? 1 : 2;
-    g_dev_sms[dev] = sms;
+  int ok = g_dev_ok[dev].load();
+  if (ok == 0) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    ok = g_dev_ok[dev].load();
+    if (ok == 0) {
+      int major = 0, sms = 0;
+      cudaError_t a = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      if (a == cudaSuccess) a = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (a != cudaSuccess) return cuda_fail("cudaDeviceGetAttribute", a);
+      g_dev_sms[dev].store(sms);   // before the flag: sm_count() may read it next
+      ok = (major == 10) ? 1 : 2;
+      g_dev_ok[dev].store(ok);
+    }
   }
-  return g_dev_ok[dev] == 1 ? SP24_OK : SP24_ERR_UNSUPPORTED;
+  return ok == 1 ? SP24_OK : SP24_ERR_UNSUPPORTED;
 }
 
 int sm_count() {
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= kMaxDevices || g_dev_sms[dev] == 0) return 148;
-  return g_dev_sms[dev];
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  const int sms = g_dev_sms[dev].load();
+  return sms > 0 ? sms : 148;
+}
+
+// One thread waits, with a bounded wait of limit_ns, on an mbarrier that
+// nothing arrives at: the wait gives up, records SP24_ERR_TIMEOUT in the
+// status word and the kernel returns normally.
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  mbar_wait_limit(&bar, 0, limit_ns);
 }
 
 }  // namespace sp24
@@ -75,6 +92,13 @@ size_t sp24_meta_bytes(int64_t N, int64_t K) {
 size_t sp24_prune_workspace_bytes(int64_t K, int mode) {
   if (K < 0) return 0;
   return mode == SP24_WANDA ? static_cast<size_t>(K) * sizeof(double) : 0;
+}
+
+sp24_status sp24_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000) return SP24_ERR_ARG;
+  SP24_TRY(check_device());
+  selftest_wait_kernel<<<1, 1, 0, as_stream(stream)>>>(static_cast<uint64_t>(limit_ns));
+  return launch_status();
 }
 
 sp24_status sp24_device_status(void* stream) {

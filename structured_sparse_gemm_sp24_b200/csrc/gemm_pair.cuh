@@ -235,16 +235,8 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
                         cudaStream_t s) {
   using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
   auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC>;
-  static uint64_t attr_set = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
-    attr_set |= bit;
-  }
+  static std::atomic<uint64_t> smem_set{0};   // one bit per device
+  SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern), C::kSmemBytes, smem_set));
   const int el = kDtype == SP24_BF16 ? 2 : 1;
   const CUtensorMapDataType dt =
       kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
@@ -304,11 +296,12 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
 // so that no pair waits for another to finish.  Every pair variant holds one
 // CTA per SM, so one query (cached per device) serves them all.
 inline sp24_status pair_capacity(int* out) {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64];   // zero-initialised (static storage)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
-  if (cache[dev & 63] > 0) {
-    *out = cache[dev & 63];
+  const int cached = cache[dev & 63].load(std::memory_order_acquire);
+  if (cached > 0) {
+    *out = cached;
     return SP24_OK;
   }
   using C = PairCfg<SP24_BF16, 256, 4, SP24_OUT_BF16, 1>;
@@ -331,7 +324,7 @@ inline sp24_status pair_capacity(int* out) {
   e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
   if (e != cudaSuccess) return cuda_fail("cudaOccupancyMaxActiveClusters", e);
   if (n < 1) return SP24_ERR_UNSUPPORTED;
-  cache[dev & 63] = n;
+  cache[dev & 63].store(n, std::memory_order_release);
   *out = n;
   return SP24_OK;
 }

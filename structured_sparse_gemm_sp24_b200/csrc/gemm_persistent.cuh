@@ -238,16 +238,8 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
                               cudaStream_t s) {
   using C = PersistCfg<kDtype, BN, STAGES, OUTK>;
   auto kern = gemm_sp_persistent<kDtype, BN, STAGES, OUTK>;
-  static uint64_t attr_set = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
-    attr_set |= bit;
-  }
+  static std::atomic<uint64_t> smem_set{0};   // one bit per device
+  SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern), C::kSmemBytes, smem_set));
   const CUtensorMapDataType ydt = OUTK == SP24_OUT_INT32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                   : OUTK == SP24_OUT_INT8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                           : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;

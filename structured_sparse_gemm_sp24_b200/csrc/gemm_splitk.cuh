@@ -273,16 +273,8 @@ sp24_status launch_gemm_cfg(const CUtensorMap& ma, const CUtensorMap& mb, const 
                             cudaStream_t s) {
   using C = GemmCfg<kDtype, BN, STAGES>;
   auto kern = gemm_sp_kernel<kDtype, BN, STAGES, SPLIT>;
-  static uint64_t attr_set = 0;   // one bit per device (devices 0..63)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
-    attr_set |= bit;
-  }
+  static std::atomic<uint64_t> smem_set{0};   // one bit per device
+  SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern), C::kSmemBytes, smem_set));
   const int64_t row_tiles = (a.n + 127) / 128;
   const int64_t tok_tiles = (a.m + BN - 1) / BN;
   if (row_tiles > 65535 || tok_tiles > 65535) return SP24_ERR_UNSUPPORTED;

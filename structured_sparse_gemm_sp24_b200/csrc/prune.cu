@@ -1080,17 +1080,10 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
                                  int n_keep, void* vals, void* meta, cudaStream_t s,
                                  const void* xc, int64_t mc) {
   auto kern = stream_kernel<kPrune, kWanda, kVals, kMaskIn>;
-  static uint64_t attr_set = 0;   // one bit per device
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-  const uint64_t bit = 1ull << (dev & 63);
-  if (!(attr_set & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kWanda ? kStreamSmemFused : kStreamSmem);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
-    attr_set |= bit;
-  }
+  static std::atomic<uint64_t> smem_set{0};   // one bit per device
+  SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern),
+                         kWanda ? kStreamSmemFused : kStreamSmem, smem_set));
+  cudaError_t e = cudaSuccess;
   const int64_t kblocks = (k + 127) / 128;
   const int64_t nchunks = ((n + 127) / 128) * kblocks;
   if (nchunks > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
@@ -1249,17 +1242,10 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
   const int64_t nvec = count / 4;
   const int ntail = static_cast<int>(count - nvec * 4);
   if (count >= kActBracketMin) {
-    static uint64_t attr_set = 0;   // one bit per device (devices 0..63)
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_fail("cudaGetDevice", cudaErrorInvalidDevice);
-    const uint64_t bit = 1ull << (dev & 63);
+    static std::atomic<uint64_t> smem_set{0};   // one bit per device
     const int sel_smem = static_cast<int>(kActSelSmemKeys * 4);
-    if (!(attr_set & bit)) {
-      const cudaError_t e = cudaFuncSetAttribute(
-          act_bracket_select, cudaFuncAttributeMaxDynamicSharedMemorySize, sel_smem);
-      if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
-      attr_set |= bit;
-    }
+    SP24_TRY(set_smem_once(reinterpret_cast<const void*>(act_bracket_select), sel_smem,
+                           smem_set));
     SP24_TRY(launch_kernel(act_sample_load, dim3(kActSampleCtas), dim3(1024), 0, s, 1, X,
                            count, ws));
     SP24_TRY(launch_kernel(act_sample_select, dim3(1), dim3(1024), 0, s, 1, count, rank, ws));

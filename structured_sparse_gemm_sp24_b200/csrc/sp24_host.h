@@ -2,6 +2,7 @@
 // checks, CUDA error mapping and the sm_100 device check.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -33,6 +34,21 @@ inline sp24_status launch_status() {
 
 // Number of SMs of the current device (cached).
 int sm_count();
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` once per device.
+// `done` holds one bit per device (0..63; check_device rejects others); two
+// threads making the first call at once may both set it, which is harmless.
+inline sp24_status set_smem_once(const void* kern, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return SP24_OK;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute", e);
+  done.fetch_or(bit, std::memory_order_release);
+  return SP24_OK;
+}
 
 // Launches every kernel of the library: programmatic stream serialization
 // (the kernel may be scheduled while the previous kernel of the stream is

@@ -65,6 +65,7 @@ SIGNATURES = {
     "sp24_prune_wanda_noalloc": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_int, _c_p, _c_p,
                                           _c_p]),
     "sp24_gemm_plan": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_p]),
+    "sp24_selftest_wait_timeout": (_c_int, [_c_i64, _c_p]),
 }
 
 
@@ -233,6 +234,13 @@ def sp24_gemm_plan(M: int, N: int, K: int, dtype: int) -> dict:
     plan = GemmPlan()
     _check(lib().sp24_gemm_plan(M, N, K, dtype, ctypes.byref(plan)), "sp24_gemm_plan")
     return plan.as_dict()
+
+
+def sp24_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launches the bounded-wait self-test (reports SP24_ERR_TIMEOUT through
+    sp24_device_status)."""
+    _check(lib().sp24_selftest_wait_timeout(limit_ns, _stream(stream)),
+           "sp24_selftest_wait_timeout")
 
 
 def sp24_device_status(stream=None) -> int:

@@ -554,6 +554,75 @@ def test_gemm_splitk_forced(split, mnk, monkeypatch):
     ok_status()
 
 
+# ------------------------------------------------------------ failure path
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert B.sp24_device_status() == B.SP24_OK
+    B.sp24_selftest_wait_timeout(20_000_000)          # 20 ms, nothing arrives
+    assert B.sp24_device_status() == B.SP24_ERR_TIMEOUT
+    assert B.sp24_device_status() == B.SP24_OK         # read and cleared
+    w = I.normal_bf16((64, 128), 1.0, seed=3)        # the library still works
+    mask = P.prune(w.cuda(), B.SP24_MAGNITUDE, 2)
+    assert np.array_equal(keep_of(mask, 128), O.prune(f64(w), O.MAGNITUDE, 2))
+    ok_status()
+    with pytest.raises(B.Sp24Error):
+        B.sp24_selftest_wait_timeout(0)
+
+
+_CONCURRENT_FIRST_CALLS = r"""
+import sys, threading, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+from oracle import sp24_oracle as O
+from structured_sparse_gemm_sp24_b200 import inputs as I, pipeline as P, sp24 as B
+torch.cuda.set_device(0)
+B.lib()
+shapes = [(2500, 2056, 400), (16, 392, 1024), (300, 24, 128), (4099, 1032, 784)]
+data, out, err = [], [None] * 4, []
+for i, (m, n, k) in enumerate(shapes):
+    W = I.normal_bf16((n, k), 1.0, seed=100 + i)
+    X = I.normal_bf16((m, k), 1.0, seed=200 + i)
+    Wd = W.cuda()
+    mask = P.prune(Wd, B.SP24_MAGNITUDE, 2)
+    vals, meta = P.compress(Wd, mask, B.SP24_BF16)
+    data.append((W, X, X.cuda(), vals, meta, n))
+torch.cuda.synchronize()
+go = threading.Barrier(4)
+def run(i):
+    try:
+        W, X, Xd, vals, meta, n = data[i]
+        st = torch.cuda.Stream()
+        with torch.cuda.stream(st):
+            go.wait()          # first GEMM launches of the process, all at once
+            y = P.gemm(Xd, vals, meta, n)
+        st.synchronize()
+        out[i] = y
+    except Exception as e:
+        err.append(repr(e))
+ts = [threading.Thread(target=run, args=(i,)) for i in range(4)]
+[t.start() for t in ts]; [t.join() for t in ts]
+assert not err, err
+assert B.sp24_device_status() == B.SP24_OK
+for i, (W, X, _, _, _, n) in enumerate(data):
+    keep = O.prune(W.double().numpy(), O.MAGNITUDE, 2)
+    v, mt = O.compress(W.double().numpy(), keep)
+    yr, ar = O.gemm(X.double().numpy(), v, mt, W.shape[1])
+    d = np.abs(out[i].double().cpu().numpy() - yr)
+    assert (d <= 8e-3 * ar + 1e-30).all(), i
+print("ok")
+"""
+
+
+def test_concurrent_first_calls_from_host_threads():
+    # a fresh process, so the per-device kernel attributes and plan caches are
+    # set up by four threads racing on their first GEMM launches
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _CONCURRENT_FIRST_CALLS, root],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stderr[-2000:]
+
+
 # ------------------------------------------------------------ launch plans
 def test_gemm_plan_families(monkeypatch):
     monkeypatch.delenv("SP24_GEMM_IMPL", raising=False)
