@@ -352,6 +352,23 @@ def count_step_kernels(runner):
         return None
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The maximum of a per-rank time over all ranks (every rank calls it at the
+    same point; all_reduce MAX), or the value itself in a single process."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, steps: int, flops_per_step: float, total_ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank runs `steps` steps of
+    its own replica; the job takes the slowest rank's time."""
+    return world * steps * flops_per_step / (total_ms * 1e-3) / 1e12
+
+
 def time_e2e(runner, steps, device):
     """Same step through host buffers: pinned H2D copies of the step's inputs and
     a D2H copy of Y inside the timed region."""
@@ -510,22 +527,14 @@ def main(argv=None):
         tot, prune, comp, gemm = time_steps(runner, args.steps, flush, stream,
                                             use_graph=not args.no_graph)
     barrier()
-    total_ms = sum(tot)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(tot), device)
     ms_per_step = total_ms / args.steps
-    value = world * args.steps * runner.flops() / (total_ms * 1e-3) / 1e12
+    value = job_tflops(world, args.steps, runner.flops(), total_ms)
 
-    e2e_ms, h2d, d2h = time_e2e(runner, max(3, min(args.steps, 50)), device)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * runner.flops() / (e2e_ms * 1e-3) / 1e12
+    e2e_steps = max(3, min(args.steps, 50))
+    e2e_ms, h2d, d2h = time_e2e(runner, e2e_steps, device)
+    e2e_ms = max_over_ranks(e2e_ms, device)
+    e2e_value = job_tflops(world, 1, runner.flops(), e2e_ms)
     if B.sp24_device_status() != B.SP24_OK:
         raise SystemExit("device status not OK after timing")
 
