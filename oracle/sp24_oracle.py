@@ -315,6 +315,23 @@ def gemm_int8_acc(xq: np.ndarray, vals_q: np.ndarray, meta: np.ndarray, k: int) 
     return acc
 
 
+def fake_quant(w: np.ndarray, keep: np.ndarray, s_w: np.ndarray) -> np.ndarray:
+    """Forward fake-quantisation of the kept weights for Sparse-QAT
+    ([Ampere-sparsity] "PTQ and QAT": in the forward pass the weights are
+    quantised to int8 and dequantised back to floating point to simulate the
+    quantisation; the STE backward and training are not part of this).
+
+    Kept position: bf16_rne(float32(q) * s_w[n]) with q = quantize(w, s_w[n])
+    (the same per-channel scale as the int8 inference path); dropped position:
+    +0.  Returns bf16 bit patterns [N, K]."""
+    w = np.asarray(w, dtype=np.float64)
+    keep = np.asarray(keep, dtype=bool)
+    s = np.asarray(s_w, dtype=np.float32)[:, None]
+    q = quantize(w.astype(np.float32), s).astype(np.float32)
+    out = bf16_rne((q * s).astype(np.float32))
+    return np.where(keep, out, np.uint16(0)).astype(np.uint16)
+
+
 def dequant_bf16(acc: np.ndarray, s_x, s_w: np.ndarray) -> np.ndarray:
     """y = bf16_rne(float32(acc) * (s_x * s_w[n])), every step float32 RN.
     Returns bf16 bit patterns [M, N]."""

@@ -390,3 +390,32 @@ def test_wanda_prune_uses_input_columns():
     keep = O.prune(w, O.WANDA, 2, xc=xc)
     assert keep[:, :4].astype(int).tolist() == [[0, 0, 1, 1]] * 2
     assert keep[:, 4:].astype(int).tolist() == [[1, 1, 0, 0]] * 2
+
+
+# --------------------------------------------------------- Sparse-QAT fake quant
+def _bits_to_f32(b):
+    return (np.asarray(b, dtype=np.uint32) << 16).view(np.float32)
+
+
+def test_fake_quant_round_trips_exact_multiples():
+    # w = k * s with s a power of two and |k| <= 127: quantise -> dequantise
+    # must give w back exactly (k * s is exact in bf16 for |k| < 256)
+    s = np.float32(2.0 ** -5)
+    k = np.arange(-127, 128, dtype=np.float64)
+    w = (k * float(s))[None, :].repeat(2, 0)
+    w = np.concatenate([w, np.zeros((2, 1))], axis=1)          # K = 256
+    keep = np.ones_like(w, dtype=bool)
+    got = _bits_to_f32(O.fake_quant(w, keep, np.array([s, s], dtype=np.float32)))
+    assert np.array_equal(got.astype(np.float64), w)
+
+
+def test_fake_quant_clamps_ties_and_drops():
+    s = np.float32(0.25)
+    w = np.array([[200 * 0.25, -200 * 0.25, 2.5 * 0.25, 3.5 * 0.25, -2.5 * 0.25, 0.5 * 0.25,
+                   1.0, 1.0]])
+    keep = np.array([[1, 1, 1, 1, 1, 1, 0, 1]], dtype=bool)
+    got = _bits_to_f32(O.fake_quant(w, keep, np.array([s], dtype=np.float32)))[0]
+    # clamp to +-127 s; half-integer quotients round to even: 2.5 -> 2, 3.5 -> 4,
+    # -2.5 -> -2, 0.5 -> 0; a dropped position is +0
+    assert list(got) == [127 * 0.25, -127 * 0.25, 0.5, 1.0, -0.5, 0.0, 0.0, 1.0]
+    assert O.fake_quant(w, keep, np.array([s], dtype=np.float32))[0, 6] == 0   # +0 bits
