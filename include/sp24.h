@@ -153,6 +153,22 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage,
 sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x,
                           int8_t* Xq, void* stream);
 
+/* Forward fake-quantisation of the masked weights for quantisation-aware
+ * training ([Ampere-sparsity] "PTQ and QAT": the forward pass quantises the
+ * weights to int8 and dequantises them back to floating point; the STE
+ * backward pass and training are not part of this library):
+ *   kept position:    W_fq = bf16_rne(float(q) * s_w[n]),
+ *                     q = clamp(rint(W / s_w[n]), -127, 127), float32 divide,
+ *                     round half to even (the code sp24_compress(SP24_INT8)
+ *                     stores for the same W, mask and s_w);
+ *   dropped position: W_fq = +0.
+ *   W, W_fq: bf16 [N][K].  mask: sp24_mask_bytes(N, K) bytes.  s_w: float32
+ *   [N] (from sp24_wscale).
+ * Rules: N >= 0, K % 8 == 0; W and W_fq 16-byte aligned. */
+sp24_status sp24_fake_quant(const void* W, const uint8_t* mask, int64_t N, int64_t K,
+                            const float* s_w, void* W_fq, void* stream);
+
+
 /* ---------------------------------------------------------- compression */
 
 /* Compression ([Ampere-sparsity] Figure 1; [Orin ch.7] 2.1 Step 2): for each

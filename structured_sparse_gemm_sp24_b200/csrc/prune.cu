@@ -1028,6 +1028,46 @@ __global__ void quantize_tail(const float* __restrict__ x, int64_t start, int64_
 }
 
 
+// ------------------------------------------- Sparse-QAT fake quantisation
+// [Ampere-sparsity] "PTQ and QAT": the forward pass of quantisation-aware
+// training quantises the weights to int8 and dequantises them back.  For the
+// masked weights: kept -> bf16(float(q) * s_w[row]) with q the int8 code of
+// the inference quantiser (q8), dropped -> +0.  One thread per 8 weights of a
+// row (16-byte load and store; bit j of the mask byte is weight j).
+__device__ __forceinline__ uint32_t fake_quant_one(uint32_t bits16, bool kept, float s, float rs) {
+  if (!kept) return 0u;
+  const int q = static_cast<int8_t>(q8(__uint_as_float(bits16 << 16), s, rs) & 0xFFu);
+  const float f = __fmul_rn(__int2float_rn(q), s);
+  return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(f)));
+}
+
+__global__ void __launch_bounds__(256) fake_quant_kernel(const uint4* __restrict__ w,
+                                                         const uint8_t* __restrict__ mask,
+                                                         const float* __restrict__ s_w, int64_t n,
+                                                         int64_t kvec, uint4* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  for (int64_t row = blockIdx.y; row < n; row += gridDim.y) {
+    const float s = __ldg(s_w + row);
+    const float rs = __frcp_rn(s);
+    for (int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; v < kvec;
+         v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t i = row * kvec + v;
+      const uint4 q = __ldcs(w + i);
+      const uint32_t m = __ldg(mask + i);
+      const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = fake_quant_one(words[e] & 0xFFFFu, (m >> (2 * e)) & 1u, s, rs);
+        const uint32_t hi = fake_quant_one(words[e] >> 16, (m >> (2 * e + 1)) & 1u, s, rs);
+        o[e] = lo | (hi << 16);
+      }
+      __stcs(out + i, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
 // ------------------------------------------- Wanda prune without allocation
 // For callers that may not allocate device memory (see sp24_prune_wanda_noalloc
 // in include/sp24.h): the float64 column norms live in this file-scope array
@@ -1266,6 +1306,22 @@ sp24_status sp24_act_scale(const float* X, int64_t count, double coverage, float
     hi_mask |= ((1u << bitsv[p]) - 1u) << shifts[p];
   }
   return SP24_OK;
+}
+
+sp24_status sp24_fake_quant(const void* W, const uint8_t* mask, int64_t N, int64_t K,
+                            const float* s_w, void* W_fq, void* stream) {
+  if (N < 0 || K < 0) return SP24_ERR_ARG;
+  if (N == 0 || K == 0) return SP24_OK;
+  if (!W || !mask || !s_w || !W_fq) return SP24_ERR_ARG;
+  if (K % 8 != 0 || !aligned16(W) || !aligned16(W_fq)) return SP24_ERR_ALIGN;
+  SP24_TRY(check_device());
+  const int64_t kvec = K / 8;
+  const int64_t bx = (kvec + 255) / 256;
+  const unsigned gx = static_cast<unsigned>(bx < 64 ? bx : 64);
+  const unsigned gy = static_cast<unsigned>(N < 65535 ? N : 65535);
+  return launch_kernel(fake_quant_kernel, dim3(gx, gy), dim3(256), 0, as_stream(stream), 1,
+                       static_cast<const uint4*>(W), mask, s_w, N, kvec,
+                       static_cast<uint4*>(W_fq));
 }
 
 sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x, int8_t* Xq,

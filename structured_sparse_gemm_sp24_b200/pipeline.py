@@ -96,3 +96,10 @@ def gemm(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, N: int,
         out = torch.empty((M, N), dtype=odt, device=X.device)
     _b.sp24_gemm(X, vals, meta, N, dtype, s_x, s_w, out_kind, s_y, out)
     return out
+
+
+def fake_quant(W: torch.Tensor, mask: torch.Tensor, s_w: torch.Tensor) -> torch.Tensor:
+    """Sparse-QAT forward fake-quantisation of W under `mask` with scales s_w."""
+    out = torch.empty_like(W)
+    _b.sp24_fake_quant(W, mask, s_w, out)
+    return out

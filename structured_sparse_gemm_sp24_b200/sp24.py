@@ -66,6 +66,7 @@ SIGNATURES = {
                                           _c_p]),
     "sp24_gemm_plan": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_p]),
     "sp24_selftest_wait_timeout": (_c_int, [_c_i64, _c_p]),
+    "sp24_fake_quant": (_c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p]),
 }
 
 
@@ -234,6 +235,13 @@ def sp24_gemm_plan(M: int, N: int, K: int, dtype: int) -> dict:
     plan = GemmPlan()
     _check(lib().sp24_gemm_plan(M, N, K, dtype, ctypes.byref(plan)), "sp24_gemm_plan")
     return plan.as_dict()
+
+
+def sp24_fake_quant(W: torch.Tensor, mask: torch.Tensor, s_w: torch.Tensor,
+                    W_fq: torch.Tensor, stream=None) -> None:
+    N, K = W.shape
+    _check(lib().sp24_fake_quant(_ptr(W), _ptr(mask), N, K, _ptr(s_w), _ptr(W_fq),
+                                 _stream(stream)), "sp24_fake_quant")
 
 
 def sp24_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

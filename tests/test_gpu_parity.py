@@ -554,6 +554,25 @@ def test_gemm_splitk_forced(split, mnk, monkeypatch):
     ok_status()
 
 
+# ------------------------------------------------------ Sparse-QAT fake quant
+@pytest.mark.parametrize("case", ["int8_workload", "ragged_3of4"])
+def test_fake_quant_matches_oracle(case):
+    if case == "int8_workload":
+        W = I.int8_long_tail().W                     # 4096 x 4096, 1 % long tail
+        n_keep = 2
+    else:
+        W = I.normal_bf16((130, 264), 0.02, seed=81)
+        n_keep = 3
+    Wd = W.cuda()
+    mask = P.prune(Wd, B.SP24_MAGNITUDE, n_keep)
+    s_w = P.wscale(Wd, mask)
+    got = P.fake_quant(Wd, mask, s_w)
+    ok_status()
+    keep = O.prune(f64(W), O.MAGNITUDE, n_keep)
+    ref = O.fake_quant(f64(W), keep, O.channel_scales(f64(W), keep))
+    assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+
+
 # ------------------------------------------------------------ failure path
 def test_bounded_wait_reports_timeout_and_context_survives():
     assert B.sp24_device_status() == B.SP24_OK
