@@ -44,6 +44,9 @@ Readings taken where the pages are silent or contradict one another:
   scale is the nearest-rank ``coverage`` quantile of |v| divided by 127; a
   zero quantile gives scale 1.  Dequantisation is done in float32 in the order
   c = s_x * s_w[n]; f = float(acc); y = bf16_rne(f * c).
+* Channel permutation search ([Orin ch.7] 3.1 and 6.3 give only the goal):
+  the objective, the greedy exchange rule and the integer scores it compares
+  are stated at that section below.
 
 Parity pins for every function here are in tests/test_oracle_pins.py.
 """
@@ -345,3 +348,161 @@ def requant_int8(acc: np.ndarray, s_x, s_w: np.ndarray, s_y) -> np.ndarray:
     c = (np.float32(s_x) * np.asarray(s_w, dtype=np.float32)).astype(np.float32)
     f = (np.asarray(acc, dtype=np.int64).astype(np.float32) * c[None, :]).astype(np.float32)
     return quantize(f, np.float32(s_y))
+
+
+# ---------------------------------------------------------------------------
+# f2  channel permutation search before masking
+#     [Orin ch.7] 3.1 (workflow step 2: search a channel order before the
+#     mask is made) and 6.3 (gather the large weights into the same block)
+# ---------------------------------------------------------------------------
+# Readings (the pages name the goal, not an algorithm):
+# * A permutation pi of the K input channels reorders the columns of W (and
+#   the same columns of X, so Y is unchanged); the groups of 4 are then
+#   pi[0:4], pi[4:8], ...  The objective is the kept score: over every row and
+#   every group, the sum of the n_keep largest scores.
+# * The search is greedy pairwise swapping: among all pairs of channels that
+#   sit in different groups, exchange the pair whose exchange raises the kept
+#   score the most; ties go to the pair whose smaller channel index is
+#   smallest, then whose larger index is smallest; stop when no exchange
+#   raises it or after max_swaps exchanges.
+# * So that every comparison is exact, the search runs on integer scores
+#   q = rint(s / s_max * 2**24) (float64 divide, round half to even), s as in
+#   scores(); a non-finite s counts as 0 and s_max = 0 gives q = 0.
+PERM_SCALE = 2.0 ** 24
+PERM_NO_PAIR = np.iinfo(np.int64).min   # swap_gains entry for a same-group pair
+
+
+def permutation_scores(w: np.ndarray, mode: str,
+                       norms: Optional[np.ndarray] = None) -> np.ndarray:
+    """Integer scores q [N, K] (int64) that the permutation search compares."""
+    s = scores(w, mode, norms)
+    s = np.where(np.isfinite(s), s, 0.0)
+    smax = float(s.max()) if s.size else 0.0
+    if smax == 0.0:
+        return np.zeros(s.shape, dtype=np.int64)
+    return np.rint(s / smax * PERM_SCALE).astype(np.int64)
+
+
+def _top_sum(groups: np.ndarray, n_keep: int) -> np.ndarray:
+    """Sum of the n_keep largest entries along the last axis (size 4)."""
+    return np.sort(groups, axis=-1)[..., 4 - n_keep:].sum(axis=-1)
+
+
+def kept_score(q: np.ndarray, perm: np.ndarray, n_keep: int) -> int:
+    """Objective of the permutation search: sum over rows and groups of
+    q[:, perm] of the n_keep largest entries of each group of 4."""
+    q = np.asarray(q, dtype=np.int64)
+    n, k = q.shape
+    g = q[:, np.asarray(perm)].reshape(n, k // 4, 4)
+    return int(_top_sum(g, n_keep).sum())
+
+
+def swap_gain(q: np.ndarray, perm: np.ndarray, a: int, b: int, n_keep: int) -> Optional[int]:
+    """Change of kept_score when channels a and b trade places, or None when
+    they sit in the same group.  Only the two groups involved change."""
+    perm = np.asarray(perm)
+    pos = np.empty_like(perm)
+    pos[perm] = np.arange(perm.size)
+    ga, gb = pos[a] // 4, pos[b] // 4
+    if ga == gb:
+        return None
+    old_a = q[:, perm[4 * ga:4 * ga + 4]]
+    old_b = q[:, perm[4 * gb:4 * gb + 4]]
+    new_a = old_a.copy()
+    new_a[:, pos[a] % 4] = q[:, b]
+    new_b = old_b.copy()
+    new_b[:, pos[b] % 4] = q[:, a]
+    return int((_top_sum(new_a, n_keep) + _top_sum(new_b, n_keep)
+                - _top_sum(old_a, n_keep) - _top_sum(old_b, n_keep)).sum())
+
+
+def swap_gains(q: np.ndarray, perm: np.ndarray, n_keep: int) -> np.ndarray:
+    """swap_gain for every ordered pair as a [K, K] int64 matrix; pairs in the
+    same group (and a == b) hold PERM_NO_PAIR.  Same arithmetic as swap_gain,
+    evaluated for all partners b of one channel a at a time."""
+    q = np.asarray(q, dtype=np.int64)
+    perm = np.asarray(perm)
+    n, k = q.shape
+    pos = np.empty_like(perm)
+    pos[perm] = np.arange(k)
+    group = pos // 4
+    members = perm.reshape(k // 4, 4)
+    kept = _top_sum(q[:, members], n_keep)            # [N, G] kept score per group
+    out = np.full((k, k), PERM_NO_PAIR, dtype=np.int64)
+    for a in range(k):
+        bs = np.flatnonzero(group != group[a])
+        if bs.size == 0:
+            continue
+        new_a = np.repeat(q[:, members[group[a]]][:, None, :], bs.size, axis=1)
+        new_a[:, :, pos[a] % 4] = q[:, bs]
+        new_b = q[:, members[group[bs]]]              # [N, len(bs), 4]
+        new_b[:, np.arange(bs.size), pos[bs] % 4] = q[:, a][:, None]
+        gain = (_top_sum(new_a, n_keep).sum(axis=0) + _top_sum(new_b, n_keep).sum(axis=0)
+                - kept[:, group[a]].sum() - kept[:, group[bs]].sum(axis=0))
+        out[a, bs] = gain
+    return out
+
+
+
+def permutation_search(q: np.ndarray, n_keep: int, max_swaps: int):
+    """Greedy pairwise channel swapping (readings above).
+
+    Returns (perm, swaps, before, after): perm[j] is the channel placed at
+    position j, swaps the number of exchanges made, before/after the kept
+    score of the identity and of perm."""
+    if n_keep not in (2, 3):
+        raise ValueError("n_keep must be 2 or 3")
+    q = np.asarray(q, dtype=np.int64)
+    n, k = q.shape
+    if k % 4:
+        raise ValueError("K must be a multiple of 4")
+    perm = np.arange(k)
+    before = kept_score(q, perm, n_keep)
+    swaps = 0
+    while swaps < max_swaps:
+        gains = swap_gains(q, perm, n_keep)
+        best = 0
+        pair = None
+        for a in range(k):                 # first strict maximum in (a, b) order
+            for b in range(a + 1, k):
+                if gains[a, b] != PERM_NO_PAIR and gains[a, b] > best:
+                    best, pair = int(gains[a, b]), (a, b)
+        if pair is None:
+            break
+        a, b = pair
+        ia, ib = int(np.flatnonzero(perm == a)[0]), int(np.flatnonzero(perm == b)[0])
+        perm[ia], perm[ib] = b, a
+        swaps += 1
+    return perm, swaps, before, kept_score(q, perm, n_keep)
+
+
+def _partitions(cols):
+    """Every split of the tuple `cols` into unordered groups of 4."""
+    if not cols:
+        yield []
+        return
+    first, rest = cols[0], cols[1:]
+    for i in range(len(rest)):
+        for j in range(i + 1, len(rest)):
+            for l in range(j + 1, len(rest)):
+                group = (first, rest[i], rest[j], rest[l])
+                left = tuple(c for t, c in enumerate(rest) if t not in (i, j, l))
+                for tail in _partitions(left):
+                    yield [group] + tail
+
+
+def best_kept_score_bruteforce(q: np.ndarray, n_keep: int) -> int:
+    """Largest kept_score over every grouping of the K channels (tiny K
+    only: K = 8 has 35 groupings, K = 12 has 5775)."""
+    q = np.asarray(q, dtype=np.int64)
+    k = q.shape[1]
+    best = None
+    for groups in _partitions(tuple(range(k))):
+        v = kept_score(q, np.array([c for g in groups for c in g]), n_keep)
+        best = v if best is None else max(best, v)
+    return best
+
+
+def permute_columns(a: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    """A[:, perm]: column j of the result is column perm[j] of A."""
+    return np.asarray(a)[:, np.asarray(perm)]

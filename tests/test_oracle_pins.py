@@ -419,3 +419,128 @@ def test_fake_quant_clamps_ties_and_drops():
     # -2.5 -> -2, 0.5 -> 0; a dropped position is +0
     assert list(got) == [127 * 0.25, -127 * 0.25, 0.5, 1.0, -0.5, 0.0, 0.0, 1.0]
     assert O.fake_quant(w, keep, np.array([s], dtype=np.float32))[0, 6] == 0   # +0 bits
+
+
+# ------------------------------------------------- channel permutation search
+# [Orin ch.7] 3.1 step 2 and 6.3: search a channel order before masking so
+# that large weights share groups.  The greedy rule and the integer scores are
+# readings (see the oracle); the hand-derived cases below follow them step by
+# step, and brute force over every grouping bounds the result.
+
+def test_perm_scores_scale_round_half_even_and_edges():
+    big = float(2 ** 24)
+    q = O.permutation_scores(np.array([[big, -big / 2, 0.5, 1.5, 2.5, -0.0, 3.0, 0.0]]),
+                             O.MAGNITUDE)
+    # s / s_max * 2^24 = s here; 0.5 -> 0, 1.5 -> 2, 2.5 -> 2 (half to even)
+    assert q.tolist() == [[2 ** 24, 2 ** 23, 0, 2, 2, 0, 3, 0]]
+    assert not O.permutation_scores(np.zeros((3, 8)), O.MAGNITUDE).any()
+    q = O.permutation_scores(np.array([[np.nan, np.inf, 4.0, -2.0]]), O.MAGNITUDE)
+    assert q.tolist() == [[0, 0, 2 ** 24, 2 ** 23]]
+    q = O.permutation_scores(np.array([[1.0, -1.0, 2.0, 1.0]]), O.WANDA,
+                             norms=np.array([4.0, 2.0, 1.0, 0.0]))
+    assert q.tolist() == [[2 ** 24, 2 ** 23, 2 ** 23, 0]]
+
+
+def test_perm_hand_example_two_of_four():
+    # One row [9 9 9 9 | 0 0 0 0].  Step 1: every (a in 0..3, b in 4..7)
+    # moves a 9 into the empty group, gain 9; the lowest pair (0, 4) wins.
+    # Step 2: groups {0,9,9,9 | 9,0,0,0}; moving one more 9 across gains 9
+    # ((1, 5) is the lowest such pair); swapping 9 for 9 gains 0 and moving
+    # the 9 back loses 9.  Step 3: every swap gains <= 0, stop.
+    q = O.permutation_scores(np.array([[9, 9, 9, 9, 0, 0, 0, 0]], float), O.MAGNITUDE)
+    perm, swaps, before, after = O.permutation_search(q, 2, 100)
+    assert perm.tolist() == [4, 5, 2, 3, 0, 1, 6, 7]
+    assert (swaps, before, after) == (2, 2 * 2 ** 24, 4 * 2 ** 24)
+    perm1, swaps1, _, after1 = O.permutation_search(q, 2, 1)
+    assert perm1.tolist() == [4, 1, 2, 3, 0, 5, 6, 7] and (swaps1, after1) == (1, 3 * 2 ** 24)
+    assert O.best_kept_score_bruteforce(q, 2) == after
+
+
+def test_perm_hand_example_three_of_four():
+    # One row [4 3 2 1 | 8 7 6 5], keep 3: kept 9 + 21 = 30.  The best
+    # grouping drops the two smallest values (1 and 2) from different groups:
+    # 36 - 3 = 33, so no swap gains more than 3.  Pairs (0, *) gain 1 and
+    # (1, *) gain 2; (2, 4) gives {4,3,8,1 | 2,7,6,5} = 15 + 18 = 33, the
+    # first pair with gain 3.  Units: q = v * 2^24 / 8 = v * 2^21.
+    q = O.permutation_scores(np.array([[4, 3, 2, 1, 8, 7, 6, 5]], float), O.MAGNITUDE)
+    perm, swaps, before, after = O.permutation_search(q, 3, 100)
+    assert perm.tolist() == [0, 1, 4, 3, 2, 5, 6, 7]
+    assert (swaps, before, after) == (1, 30 * 2 ** 21, 33 * 2 ** 21)
+    assert O.best_kept_score_bruteforce(q, 3) == 33 * 2 ** 21
+    g = O.swap_gains(q, np.arange(8), 3)
+    assert [g[0, b] for b in range(4, 8)] == [2 ** 21] * 4
+    assert [g[1, b] for b in range(4, 8)] == [2 * 2 ** 21] * 4
+    assert g[2, 4] == 3 * 2 ** 21
+
+
+def test_perm_pages_row_is_already_optimal():
+    # The 1x4 row [0.9 0.1 0.9 0.1] that [Orin ch.7] 3.1 uses to motivate the
+    # permutation already keeps both 0.9 under the keep-the-largest rule; no
+    # exchange can raise the kept score, so the search leaves the order alone.
+    q = O.permutation_scores(np.array([[0.9, 0.1, 0.9, 0.1] * 2]), O.MAGNITUDE)
+    perm, swaps, before, after = O.permutation_search(q, 2, 100)
+    assert perm.tolist() == list(range(8)) and swaps == 0 and before == after
+    assert O.best_kept_score_bruteforce(q, 2) == before
+
+
+@pytest.mark.parametrize("n_keep", [2, 3])
+def test_perm_gains_equal_full_rescore(n_keep):
+    rng = np.random.default_rng(11 + n_keep)
+    q = rng.integers(0, 6, size=(5, 12)).astype(np.int64)   # small range: many ties
+    for perm in (np.arange(12), rng.permutation(12)):
+        g = O.swap_gains(q, perm, n_keep)
+        base = O.kept_score(q, perm, n_keep)
+        pos = np.argsort(perm)
+        for a in range(12):
+            for b in range(12):
+                if pos[a] // 4 == pos[b] // 4:
+                    assert g[a, b] == O.PERM_NO_PAIR and O.swap_gain(q, perm, a, b, n_keep) is None
+                    continue
+                p2 = perm.copy()
+                p2[pos[a]], p2[pos[b]] = b, a
+                want = O.kept_score(q, p2, n_keep) - base
+                assert g[a, b] == want == O.swap_gain(q, perm, a, b, n_keep)
+
+
+def test_perm_partition_enumeration_is_complete():
+    for k, count in ((4, 1), (8, 35), (12, 5775)):
+        seen = set()
+        for groups in O._partitions(tuple(range(k))):
+            assert sorted(c for g in groups for c in g) == list(range(k))
+            seen.add(frozenset(frozenset(g) for g in groups))
+        # K! / ((4!)^(K/4) * (K/4)!) groupings, each produced once
+        assert len(seen) == count == math.factorial(k) // (
+            math.factorial(4) ** (k // 4) * math.factorial(k // 4))
+
+
+@pytest.mark.parametrize("n_keep", [2, 3])
+@pytest.mark.parametrize("k", [8, 12])
+def test_perm_search_is_a_local_optimum_under_the_bruteforce_bound(n_keep, k):
+    rng = np.random.default_rng(100 * k + n_keep)
+    for trial in range(3):
+        w = rng.standard_normal((4, k)) * rng.uniform(0.2, 3.0, size=k)
+        q = O.permutation_scores(w, O.MAGNITUDE)
+        perm, swaps, before, after = O.permutation_search(q, n_keep, 1000)
+        assert sorted(perm.tolist()) == list(range(k))
+        assert before == O.kept_score(q, np.arange(k), n_keep)
+        assert after == O.kept_score(q, perm, n_keep)
+        assert before + swaps <= after <= O.best_kept_score_bruteforce(q, n_keep)
+        pos = np.argsort(perm)
+        for a in range(k):                        # no single exchange improves
+            for b in range(a + 1, k):
+                if pos[a] // 4 != pos[b] // 4:
+                    p2 = perm.copy()
+                    p2[pos[a]], p2[pos[b]] = b, a
+                    assert O.kept_score(q, p2, n_keep) <= after
+
+
+def test_perm_columns_leave_the_product_unchanged():
+    # The exchange is an equivalent transform: permuting the same input
+    # channels of X and W leaves Y = X W^T unchanged (exact in integers).
+    rng = np.random.default_rng(5)
+    x = rng.integers(-9, 10, size=(6, 16))
+    w = rng.integers(-9, 10, size=(5, 16))
+    perm = rng.permutation(16)
+    xp, wp = O.permute_columns(x, perm), O.permute_columns(w, perm)
+    assert (xp @ wp.T == x @ w.T).all()
+    assert (xp[:, np.argsort(perm)] == x).all()
