@@ -470,6 +470,48 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------- main
+def run_permute_search(args):
+    """Times the channel permutation search on the workload's weight shape
+    (channel-scaled synthetic weights, magnitude scores, keep 2 of 4): CUDA
+    events on the stream around the whole blocking call, set-up included.
+    Prints one JSON line."""
+    torch.cuda.set_device(0)
+    device = torch.device("cuda", 0)
+    B.lib()
+    from structured_sparse_gemm_sp24_b200 import pipeline as P
+    wl = I.by_name(args.workload)
+    n, k = wl.W.shape
+    w = I.channel_scaled_bf16((n, k), 0.02, 5).to(device)
+    limit = args.permute_max_swaps if args.permute_max_swaps is not None else 64 * k
+    for _ in range(args.warmup):
+        perm, res = P.permute_search(w, 2, None, limit)
+    times = []
+    for _ in range(args.steps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        perm, res = P.permute_search(w, 2, None, limit)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    if B.sp24_device_status() != B.SP24_OK:
+        raise SystemExit("device status not OK after the permutation search")
+    ms = statistics.median(times)
+    swaps = int(res["swaps"])
+    line = {
+        "metric": "channel permutation search time", "value": round(ms, 3), "unit": "ms",
+        "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "dtype": "int32/int64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}_weight_permute", "N": n, "K": k, "n_keep": 2,
+                   "max_swaps": limit, "weights": "channel_scaled_bf16 sigma 0.02 seed 5"},
+        "swaps": swaps, "us_per_swap": round(1e3 * ms / max(swaps, 1), 2),
+        "kept_gain_pct": round(100.0 * (res["kept_after"] / max(res["kept_before"], 1) - 1), 4),
+        "converged": swaps < limit,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -481,7 +523,12 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-graph", action="store_true",
                     help="time plain launches instead of a CUDA-graph replay of the step")
+    ap.add_argument("--permute-search", action="store_true",
+                    help="time the channel permutation search on the workload's weight shape")
+    ap.add_argument("--permute-max-swaps", type=int, default=None)
     args = ap.parse_args(argv)
+    if args.permute_search:
+        return run_permute_search(args)
     args.warmup = max(3, args.warmup)
     if args.impl == "reference":
         return run_reference(args)

@@ -6,7 +6,8 @@
  *   compress W + mask (+ INT8 scales)        -> values + metadata (tcgen05 operand layout)
  *   gemm     X, values, metadata (+ scales)  -> Y = X * W'^T
  * plus the INT8 calibration helpers (per-channel / per-tensor scales,
- * activation quantisation) and status queries.
+ * activation quantisation), the channel permutation search that may precede
+ * pruning, and status queries.
  *
  * Sources ("pages") are cited by title and section:
  *   [Ampere-sparsity] NVIDIA x Tencent MLPD article on Ampere fine-grained
@@ -22,13 +23,14 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Pointers named W, X, Xc, mask*, vals, meta, norms, s_*, Y and workspace are
+ * - Pointers named W, X, Xc, A*, mask*, vals, meta, norms, perm, s_*, Y and workspace are
  *   DEVICE pointers owned by the caller; the library never allocates, frees or
  *   keeps them.  Matrices are row-major and densely packed (row stride = number
  *   of columns).  Every device pointer must be 16-byte aligned (cudaMalloc
  *   gives 256) or the call returns SP24_ERR_ALIGN.
  * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
- *   Every call only enqueues work; it does not synchronise.
+ *   Every call only enqueues work; it does not synchronise, except
+ *   sp24_permute_search, which says so.
  * - Argument, size and alignment errors are detected on the host before any
  *   launch and returned synchronously; nothing is enqueued in that case.
  * - Errors found on the device (a group that does not keep exactly two
@@ -57,7 +59,8 @@ typedef enum sp24_status {
     SP24_ERR_PATTERN = 3,     /* a group of 4 does not keep exactly two positions */
     SP24_ERR_CUDA = 4,        /* a CUDA runtime call failed */
     SP24_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
-    SP24_ERR_UNSUPPORTED = 6  /* no sm_100 device, or a combination not provided */
+    SP24_ERR_UNSUPPORTED = 6, /* no sm_100 device, or a combination not provided */
+    SP24_ERR_INDEX = 7        /* a permutation entry lies outside [0, K) */
 } sp24_status;
 
 /* scoring modes for sp24_prune */
@@ -120,6 +123,62 @@ sp24_status sp24_colnorm(const void* Xc, int64_t Mc, int64_t K, double* norms,
 sp24_status sp24_prune(const void* W, int64_t N, int64_t K, const void* Xc,
                        int64_t Mc, int mode, int n_keep, const uint8_t* mask_in,
                        uint8_t* mask_out, void* workspace, void* stream);
+
+/* ------------------------------------------------- channel permutation */
+
+/* Largest K accepted by the permutation search (its gain table is K x K
+ * int64). */
+#define SP24_PERMUTE_MAX_K 65536
+
+/* Outcome of sp24_permute_search (host struct). */
+typedef struct sp24_permute_result_t {
+    int64_t swaps;        /* exchanges made */
+    int64_t kept_before;  /* kept score of the identity order (integer scores) */
+    int64_t kept_after;   /* kept score of the returned order */
+} sp24_permute_result_t;
+
+/* Scratch bytes of sp24_permute_search: 8*N*K + 8*K*K + O(N + K); 0 for
+ * arguments the search rejects. */
+size_t sp24_permute_workspace_bytes(int64_t N, int64_t K);
+
+/* Channel permutation search before masking ([Orin ch.7] 3.1 workflow step 2
+ * and 6.3: choose an order of the input channels so that large weights share
+ * groups of 4 before the mask is made).  The pages give the goal only; this
+ * library reads it as:
+ *   objective  kept score = over every row and every group of 4 consecutive
+ *              positions of W[:, perm], the sum of the n_keep largest scores;
+ *   scores     s = |w| (norms == NULL) or |w| * norms[j] (float64, the
+ *              sp24_prune Wanda score), a score that is not a finite positive
+ *              number counting as 0; compared as the integers
+ *              q = rint(s / s_max * 2^24) (float64 divide, half to even), so
+ *              every comparison below is exact;
+ *   search     greedy exchange: starting from the identity, repeatedly swap
+ *              the two channels in different groups whose swap raises the
+ *              kept score most (ties: smallest lower channel index, then
+ *              smallest upper index); stop when no swap raises it or after
+ *              max_swaps swaps.
+ *   W: bf16 [N][K].  norms: float64 [K] or NULL.
+ *   perm: int32 [K] (device, written): position j of the new order holds
+ *         channel perm[j]; apply it with sp24_permute_columns to W and to
+ *         the matching columns of X (Y is unchanged), then prune as usual.
+ *   workspace: sp24_permute_workspace_bytes(N, K) bytes (workspace_bytes
+ *         says how many the caller passes).
+ *   result: host struct, nullable.
+ * The call BLOCKS the calling thread: it synchronises `stream` between
+ * batches of steps to learn whether the search has stopped.
+ * Rules: N >= 1, 4 <= K <= SP24_PERMUTE_MAX_K, K % 4 == 0, n_keep in {2, 3},
+ * max_swaps >= 0; norms, if given, >= 0 (as sp24_colnorm writes them). */
+sp24_status sp24_permute_search(const void* W, int64_t N, int64_t K, const double* norms,
+                                int n_keep, int64_t max_swaps, int32_t* perm,
+                                void* workspace, size_t workspace_bytes,
+                                sp24_permute_result_t* result, void* stream);
+
+/* Column gather that applies a channel order: A_out[r][j] = A[r][perm[j]] for
+ * a row-major [rows][K] matrix of elem_bytes-byte elements (1, 2 or 4: int8,
+ * bf16, float32).  A and A_out must not overlap.  An entry of perm outside
+ * [0, K) writes 0 and records SP24_ERR_INDEX in the device status word. */
+sp24_status sp24_permute_columns(const void* A, int64_t rows, int64_t K, int elem_bytes,
+                                 const int32_t* perm, void* A_out, void* stream);
 
 /* --------------------------------------------------------- INT8 scales */
 
@@ -290,7 +349,7 @@ sp24_status sp24_prune_wanda_noalloc(const void* W, int64_t N, int64_t K, const 
 sp24_status sp24_selftest_wait_timeout(int64_t limit_ns, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word of the
- * current device (SP24_OK, SP24_ERR_PATTERN or SP24_ERR_TIMEOUT), or
+ * current device (SP24_OK, SP24_ERR_PATTERN, SP24_ERR_TIMEOUT or SP24_ERR_INDEX), or
  * SP24_ERR_CUDA if the stream reports a CUDA error. */
 sp24_status sp24_device_status(void* stream);
 

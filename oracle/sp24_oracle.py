@@ -367,7 +367,8 @@ def requant_int8(acc: np.ndarray, s_x, s_w: np.ndarray, s_y) -> np.ndarray:
 #   raises it or after max_swaps exchanges.
 # * So that every comparison is exact, the search runs on integer scores
 #   q = rint(s / s_max * 2**24) (float64 divide, round half to even), s as in
-#   scores(); a non-finite s counts as 0 and s_max = 0 gives q = 0.
+#   scores(); an s that is not a finite positive number counts as 0 and
+#   s_max = 0 gives q = 0.
 PERM_SCALE = 2.0 ** 24
 PERM_NO_PAIR = np.iinfo(np.int64).min   # swap_gains entry for a same-group pair
 
@@ -376,7 +377,7 @@ def permutation_scores(w: np.ndarray, mode: str,
                        norms: Optional[np.ndarray] = None) -> np.ndarray:
     """Integer scores q [N, K] (int64) that the permutation search compares."""
     s = scores(w, mode, norms)
-    s = np.where(np.isfinite(s), s, 0.0)
+    s = np.where(np.isfinite(s) & (s > 0), s, 0.0)
     smax = float(s.max()) if s.size else 0.0
     if smax == 0.0:
         return np.zeros(s.shape, dtype=np.int64)

@@ -115,6 +115,7 @@ sp24_status sp24_device_status(void* stream) {
   }
   if (word & kErrTimeoutBit) return SP24_ERR_TIMEOUT;
   if (word & kErrPatternBit) return SP24_ERR_PATTERN;
+  if (word & kErrIndexBit) return SP24_ERR_INDEX;
   return SP24_OK;
 }
 
@@ -127,6 +128,7 @@ const char* sp24_strerror(int status) {
     case SP24_ERR_CUDA: return "CUDA runtime error";
     case SP24_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     case SP24_ERR_UNSUPPORTED: return "unsupported device or argument combination";
+    case SP24_ERR_INDEX: return "a permutation entry lies outside [0, K)";
     default: return "unknown status";
   }
 }

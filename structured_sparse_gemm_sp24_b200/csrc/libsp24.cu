@@ -3,3 +3,4 @@
 #include "api.cu"
 #include "prune.cu"
 #include "gemm_sp.cu"
+#include "permute.cu"

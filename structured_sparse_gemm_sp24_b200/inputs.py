@@ -16,6 +16,10 @@ CPU so that the bytes do not depend on the device):
   from stream ``seed+3`` is multiplied by 20 in fp32 before the bf16 cast.
 * fp32 activations for the INT8 workload (to be calibrated and quantised by
   the method): ``randn`` in fp32 from stream ``seed+1``, kept in fp32.
+* channel-scaled weights (channel permutation search): ``randn * sigma`` times
+  a per-input-channel gain ``exp(spread * randn)`` from stream ``seed+4``,
+  in fp32 before the single bf16 rounding, so that some channels carry
+  larger weights than others, as trained layers do.
 
 The workload names and shapes follow the layer shapes the pages discuss:
 a BERT-base FFN fc1 (768 -> 3072), LLM projection shapes (4096 <-> 11008),
@@ -58,6 +62,15 @@ def long_tail_bf16(shape: Tuple[int, ...], sigma: float, seed: int,
     u = torch.rand(shape, generator=_gen(tail_seed), dtype=torch.float32)
     w = torch.where(u < tail_prob, w * tail_gain, w)
     return w.to(torch.bfloat16)
+
+
+def channel_scaled_bf16(shape: Tuple[int, ...], sigma: float, seed: int,
+                        spread: float = 0.5) -> torch.Tensor:
+    """[N, K] weights N(0, sigma^2) * exp(spread * g_j), g_j ~ N(0, 1) per input
+    channel j from stream ``seed + 4`` (fp32, then one bf16 rounding)."""
+    w = normal_f32(shape, sigma, seed)
+    g = torch.randn((1, shape[-1]), generator=_gen(seed + 4), dtype=torch.float32)
+    return (w * torch.exp(g * spread)).to(torch.bfloat16)
 
 
 @dataclasses.dataclass

@@ -103,3 +103,22 @@ def fake_quant(W: torch.Tensor, mask: torch.Tensor, s_w: torch.Tensor) -> torch.
     out = torch.empty_like(W)
     _b.sp24_fake_quant(W, mask, s_w, out)
     return out
+
+
+def permute_search(W: torch.Tensor, n_keep: int = 2, norms: Optional[torch.Tensor] = None,
+                   max_swaps: Optional[int] = None) -> Tuple[torch.Tensor, dict]:
+    """Channel order for W before masking (greedy exchange on the kept score).
+    Returns (perm int32 [K], {"swaps", "kept_before", "kept_after"})."""
+    N, K = W.shape
+    ws = _u8(_b.sp24_permute_workspace_bytes(N, K), W.device)
+    perm = torch.empty(K, dtype=torch.int32, device=W.device)
+    limit = 1 << 40 if max_swaps is None else max_swaps
+    res = _b.sp24_permute_search(W, norms, n_keep, limit, perm, ws)
+    return perm, res
+
+
+def permute_columns(A: torch.Tensor, perm: torch.Tensor) -> torch.Tensor:
+    """A[:, perm] (the same order applied to W and to the columns of X)."""
+    out = torch.empty_like(A)
+    _b.sp24_permute_columns(A, perm, out)
+    return out

@@ -25,6 +25,7 @@ SP24_ERR_PATTERN = 3
 SP24_ERR_CUDA = 4
 SP24_ERR_TIMEOUT = 5
 SP24_ERR_UNSUPPORTED = 6
+SP24_ERR_INDEX = 7
 SP24_MAGNITUDE = 0
 SP24_WANDA = 1
 SP24_BF16 = 0
@@ -33,6 +34,7 @@ SP24_OUT_BF16 = 0
 SP24_OUT_INT32 = 1
 SP24_OUT_INT8 = 2
 SP24_NOALLOC_MAX_K = 65536
+SP24_PERMUTE_MAX_K = 65536
 
 _c_i64 = ctypes.c_int64
 _c_p = ctypes.c_void_p
@@ -67,6 +69,10 @@ SIGNATURES = {
     "sp24_gemm_plan": (_c_int, [_c_i64, _c_i64, _c_i64, _c_int, _c_p]),
     "sp24_selftest_wait_timeout": (_c_int, [_c_i64, _c_p]),
     "sp24_fake_quant": (_c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_p, _c_p, _c_p]),
+    "sp24_permute_workspace_bytes": (_c_size, [_c_i64, _c_i64]),
+    "sp24_permute_search": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_int, _c_i64, _c_p, _c_p,
+                                     _c_size, _c_p, _c_p]),
+    "sp24_permute_columns": (_c_int, [_c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p]),
 }
 
 
@@ -80,6 +86,17 @@ class GemmPlan(ctypes.Structure):
         return {"kernel": self.kernel.decode(), "tile_tokens": self.tile_tokens,
                 "tile_channels": self.tile_channels, "split_k": self.split_k,
                 "cluster": self.cluster, "ctas": self.ctas}
+
+
+class PermuteResult(ctypes.Structure):
+    """sp24_permute_result_t."""
+    _fields_ = [("swaps", ctypes.c_int64), ("kept_before", ctypes.c_int64),
+                ("kept_after", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {"swaps": self.swaps, "kept_before": self.kept_before,
+                "kept_after": self.kept_after}
+
 
 _LIB: Optional[ctypes.CDLL] = None
 
@@ -242,6 +259,29 @@ def sp24_fake_quant(W: torch.Tensor, mask: torch.Tensor, s_w: torch.Tensor,
     N, K = W.shape
     _check(lib().sp24_fake_quant(_ptr(W), _ptr(mask), N, K, _ptr(s_w), _ptr(W_fq),
                                  _stream(stream)), "sp24_fake_quant")
+
+
+def sp24_permute_workspace_bytes(N: int, K: int) -> int:
+    return lib().sp24_permute_workspace_bytes(N, K)
+
+
+def sp24_permute_search(W: torch.Tensor, norms: Optional[torch.Tensor], n_keep: int,
+                        max_swaps: int, perm: torch.Tensor, workspace: torch.Tensor,
+                        stream=None) -> dict:
+    """Greedy channel permutation search; blocks until it has finished."""
+    N, K = W.shape
+    res = PermuteResult()
+    _check(lib().sp24_permute_search(_ptr(W), N, K, _ptr(norms), n_keep, max_swaps, _ptr(perm),
+                                     _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     ctypes.byref(res), _stream(stream)), "sp24_permute_search")
+    return res.as_dict()
+
+
+def sp24_permute_columns(A: torch.Tensor, perm: torch.Tensor, A_out: torch.Tensor,
+                         stream=None) -> None:
+    rows, K = A.shape
+    _check(lib().sp24_permute_columns(_ptr(A), rows, K, A.element_size(), _ptr(perm),
+                                      _ptr(A_out), _stream(stream)), "sp24_permute_columns")
 
 
 def sp24_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -150,3 +150,30 @@ def test_meta_layout_decoder_hand_cases():
     hw[16 * 9 + 6] = 0xCD
     canon = meta_layout.decode(hw, 128, 128, meta_layout.INT8)
     assert canon[9, 6] == 0xCD and canon.sum() == 0xCD
+
+
+def test_permute_host_validation(lib):
+    ws = lib.sp24_permute_workspace_bytes
+    # q and thr (8 N K) + gain (8 K^2) + small pieces
+    assert ws(100, 64) >= 8 * 100 * 64 + 8 * 64 * 64
+    assert ws(100, 64) < 8 * 100 * 64 + 8 * 64 * 64 + 64 * 100 + 200 * 64 + 4096
+    assert ws(0, 64) == 0 and ws(8, 6) == 0 and ws(8, 0) == 0
+    assert ws(8, B.SP24_PERMUTE_MAX_K + 4) == 0
+    f = lib.sp24_permute_search
+    big = 1 << 30
+    assert f(FAKE, 8, 16, None, 4, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ARG   # n_keep
+    assert f(FAKE, 8, 16, None, 2, -1, FAKE, FAKE, big, None, None) == B.SP24_ERR_ARG   # max_swaps
+    assert f(FAKE, 0, 16, None, 2, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ARG   # N
+    assert f(None, 8, 16, None, 2, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 8, 16, None, 2, 10, None, FAKE, big, None, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 8, 18, None, 2, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ALIGN  # K % 4
+    assert f(FAKE + 2, 8, 16, None, 2, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ALIGN
+    assert f(FAKE, 8, 16, FAKE + 8, 2, 10, FAKE, FAKE, big, None, None) == B.SP24_ERR_ALIGN
+    assert f(FAKE, 8, 16, None, 2, 10, FAKE, FAKE, ws(8, 16) - 1, None, None) == B.SP24_ERR_ARG
+    g = lib.sp24_permute_columns
+    assert g(FAKE, 4, 16, 3, FAKE, FAKE + 256, None) == B.SP24_ERR_ARG      # element size
+    assert g(FAKE, 4, 16, 2, FAKE, FAKE, None) == B.SP24_ERR_ARG            # in place
+    assert g(FAKE, -1, 16, 2, FAKE, FAKE + 256, None) == B.SP24_ERR_ARG
+    assert g(FAKE, 0, 16, 2, FAKE, FAKE + 256, None) == B.SP24_OK           # nothing to do
+    assert g(FAKE + 4, 4, 16, 2, FAKE, FAKE + 256, None) == B.SP24_ERR_ALIGN
+    assert lib.sp24_strerror(B.SP24_ERR_INDEX).decode().startswith("a permutation entry")
