@@ -19,6 +19,11 @@ namespace {
 thread_local char g_last_err[256] = "";
 }  // namespace
 
+// Status-word bit of sp24_permute_columns: a permutation entry outside
+// [0, K) (the pattern and timeout bits sit with the status word itself).
+constexpr uint32_t kErrIndexBit = 4u;
+static_assert((kErrIndexBit & (kErrPatternBit | kErrTimeoutBit)) == 0, "status bits overlap");
+
 sp24_status cuda_fail(const char* what, const char* err_name) {
   std::snprintf(g_last_err, sizeof(g_last_err), "%s: %s", what, err_name ? err_name : "?");
   return SP24_ERR_CUDA;

@@ -14,7 +14,7 @@ namespace sp24 {
 // --------------------------------------------------------------- status word
 // One word per device; kernels OR error bits into it, sp24_device_status()
 // reads and clears it.
-enum : uint32_t { kErrPatternBit = 1u, kErrTimeoutBit = 2u, kErrIndexBit = 4u };
+enum : uint32_t { kErrPatternBit = 1u, kErrTimeoutBit = 2u };
 
 // Defined here: the library is one translation unit (libsp24.cu).
 __device__ uint32_t g_status = 0;
