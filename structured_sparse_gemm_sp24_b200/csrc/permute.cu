@@ -30,7 +30,8 @@
 //                              channels of the last exchange, column-major
 //   gain     int64 [K][K]      swap gains; NO_PAIR for same-group pairs
 //   U        int64 [K]
-//   part     int64 [8][K]      M[c][b] + M[b][c] for the 8 changed channels
+//   part     int64 [2][8][K]   M[c][b] + M[b][c] for the 8 changed channels
+//                              (two buffers, alternate steps)
 //   best     int64 [K], int32 [K]  per row of gain: the largest entry and the
 //                              smallest column holding it
 //   pos      int32 [K]         inverse of perm
@@ -161,7 +162,6 @@ __global__ void __launch_bounds__(256) perm_quantize(const uint16_t* __restrict_
 // thread per group (groups are 4 consecutive channels), `rows` rows per
 // block row.
 __global__ void __launch_bounds__(256) perm_refresh_all(Ws ws, int64_t rows) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const bool live = g < ws.k / 4;
@@ -188,13 +188,13 @@ __global__ void __launch_bounds__(256) perm_refresh_all(Ws ws, int64_t rows) {
     red_add(&ws.st->before, kacc);
     red_add(&ws.st->after, kacc);
   }
+  pdl_launch_dependents();
 }
 
 // M[a][b] + M[b][a] for every pair of channels, one 64 x 64 tile of pairs
 // (upper triangle of tiles) per block over one slice of the rows.  gridDim.y
 // > 1 splits the rows and adds into a zeroed gain; otherwise it stores.
 __global__ void __launch_bounds__(256) perm_gain_full(Ws ws, int tiles, int64_t rows) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   __shared__ int4 sm[4][kRowChunk][kGainTile / 4];   // thr_A, q_A, thr_B, q_B
   int64_t idx = blockIdx.x;
@@ -267,12 +267,12 @@ __global__ void __launch_bounds__(256) perm_gain_full(Ws ws, int tiles, int64_t 
       }
     }
   }
+  pdl_launch_dependents();
 }
 
 // Finishes gain (adds U, marks same-group pairs) and the best entry of every
 // row.  One warp per row.
 __global__ void __launch_bounds__(256) perm_rowbest_full(Ws ws) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
@@ -296,13 +296,19 @@ __global__ void __launch_bounds__(256) perm_rowbest_full(Ws ws) {
       ws.best_idx[a] = bi;
     }
   }
+  pdl_launch_dependents();
 }
 
 // ------------------------------------------------------- one greedy step
+// The kernels of a step (and the longer set-up passes) signal their
+// dependents only after their main work: an early signal would let the next
+// kernel's blocks occupy SM slots while they wait.  `part` is double-buffered by the parity of the exchange
+// count: step t accumulates into part[t & 1] and, while reading it, clears
+// part[(t + 1) & 1], which step t + 1 accumulates into.
+
 // (1) Picks the best pair from the row bests, exchanges it in perm / pos and
-// clears U and part of the 8 channels of the two groups.  One block.
+// clears U of the 8 channels of the two groups.  One block.
 __global__ void __launch_bounds__(1024) perm_pick(Ws ws, int64_t max_swaps) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   State* st = ws.st;
   if (st->done) return;
@@ -342,20 +348,19 @@ __global__ void __launch_bounds__(1024) perm_pick(Ws ws, int64_t max_swaps) {
     ws.pos[b] = pa;
     st->ga = pa >> 2;
     st->gb = pb >> 2;
-    st->swaps += 1;
+    st->swaps = swaps_now + 1;
     st->after += bv;
     s_g[0] = pa >> 2;
     s_g[1] = pb >> 2;
   }
   __syncthreads();
   if (threadIdx.x < 8) ws.u[ws.perm[4 * s_g[threadIdx.x >> 2] + (threadIdx.x & 3)]] = 0;
-  for (int64_t e = threadIdx.x; e < 8 * ws.k; e += 1024) ws.part[e] = 0;
+  pdl_launch_dependents();
 }
 
 // (2) thr and U of the two exchanged groups; also the column-major copies of
 // their thr and q for step (3).  One thread per row, blockIdx.y = group.
 __global__ void __launch_bounds__(256) perm_refresh_pair(Ws ws) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   if (ws.st->done) return;
   const int slot0 = 4 * blockIdx.y;
@@ -383,14 +388,16 @@ __global__ void __launch_bounds__(256) perm_refresh_pair(Ws ws) {
     const long long s = warp_sum(uacc[i]);
     if ((threadIdx.x & 31) == 0 && s != 0) red_add(ws.u + c[i], s);
   }
+  pdl_launch_dependents();
 }
 
 // (3) part[i][b] = M[c_i][b] + M[b][c_i] for the 8 changed channels c_i and
-// every channel b: one thread per b over one slice of the rows.
+// every channel b: one thread per b over one slice of the rows.  Eight rows
+// of q and thr are loaded before they are used, to keep loads in flight.
 __global__ void __launch_bounds__(256) perm_partial(Ws ws, int64_t rows) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   if (ws.st->done) return;
+  long long* part = ws.part + (ws.st->swaps & 1) * 8 * ws.k;
   __shared__ int4 stc[kRowChunk][4];   // per row: thr of slots 0-7, q of slots 0-7
   const int64_t b = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
   const bool live = b < ws.k;
@@ -408,15 +415,25 @@ __global__ void __launch_bounds__(256) perm_partial(Ws ws, int64_t rows) {
     const int cnt = static_cast<int>(min(static_cast<int64_t>(kRowChunk), r_end - r0));
     int a32[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // 32 rows x 2 terms x 2^24 < 2^31
     if (live) {
-#pragma unroll 4
-      for (int rr = 0; rr < cnt; ++rr) {
-        const int qb = ws.q[(r0 + rr) * ws.k + b];
-        const int tb = ws.thr[(r0 + rr) * ws.k + b];
-        const int4 t0 = stc[rr][0], t1 = stc[rr][1], q0 = stc[rr][2], q1 = stc[rr][3];
-        const int tcv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-        const int qcv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      for (int rb = 0; rb < cnt; rb += 8) {
+        int qb[8], tb[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a32[i] += max(tcv[i], qb) + max(tb, qcv[i]);
+        for (int j = 0; j < 8; ++j) {
+          const bool in = rb + j < cnt;
+          const int64_t off = (r0 + rb + (in ? j : 0)) * ws.k + b;
+          qb[j] = in ? __ldg(ws.q + off) : 0;
+          tb[j] = in ? __ldg(ws.thr + off) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (rb + j >= cnt) break;
+          const int4 t0 = stc[rb + j][0], t1 = stc[rb + j][1];
+          const int4 q0 = stc[rb + j][2], q1 = stc[rb + j][3];
+          const int tcv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          const int qcv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a32[i] += max(tcv[i], qb[j]) + max(tb[j], qcv[i]);
+        }
       }
     }
 #pragma unroll
@@ -424,32 +441,40 @@ __global__ void __launch_bounds__(256) perm_partial(Ws ws, int64_t rows) {
   }
   if (live) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) red_add(ws.part + i * ws.k + b, acc[i]);
+    for (int i = 0; i < 8; ++i) red_add(part + i * ws.k + b, acc[i]);
   }
+  pdl_launch_dependents();
 }
 
 // (4) New gain rows / columns of the 8 changed channels and the row bests.
 // A row outside the two groups only needs a full rescan when its old best
-// partner is one of the 8; otherwise its other entries did not change.
+// partner is one of the 8; otherwise its other entries did not change.  Also
+// clears the other part buffer for the next step.
 __global__ void __launch_bounds__(256) perm_update(Ws ws) {
-  pdl_launch_dependents();
   pdl_wait_prior();
   if (ws.st->done) return;
   const int ga = ws.st->ga, gb = ws.st->gb;
+  const long long par = ws.st->swaps & 1;
+  const long long* part = ws.part + par * 8 * ws.k;
+  long long* next = ws.part + (par ^ 1) * 8 * ws.k;
+  for (int64_t e = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; e < 8 * ws.k;
+       e += static_cast<int64_t>(gridDim.x) * 256)
+    next[e] = 0;
   const int lane = threadIdx.x & 31;
   const int64_t warps = static_cast<int64_t>(gridDim.x) * 8;
   for (int64_t a = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); a < ws.k; a += warps) {
     const int pa = ws.pos[a];
     const int grp = pa >> 2;
     const long long ua = ws.u[a];
+    long long* row = ws.gain + a * ws.k;
     long long bv = kNoPair;
     int bi = INT_MAX;
     if (grp == ga || grp == gb) {
       const int slot = (grp == ga ? 0 : 4) + (pa & 3);
       for (int64_t b = lane; b < ws.k; b += 32) {
         long long v = kNoPair;
-        if ((ws.pos[b] >> 2) != grp) v = ua + ws.u[b] + ws.part[slot * ws.k + b];
-        ws.gain[a * ws.k + b] = v;
+        if ((ws.pos[b] >> 2) != grp) v = ua + ws.u[b] + part[slot * ws.k + b];
+        row[b] = v;
         if (v > bv) {
           bv = v;
           bi = static_cast<int>(b);
@@ -458,8 +483,8 @@ __global__ void __launch_bounds__(256) perm_update(Ws ws) {
     } else {
       if (lane < 8) {
         const int c = ws.perm[4 * (lane < 4 ? ga : gb) + (lane & 3)];
-        const long long v = ua + ws.u[c] + ws.part[lane * ws.k + a];
-        ws.gain[a * ws.k + c] = v;
+        const long long v = ua + ws.u[c] + part[lane * ws.k + a];
+        row[c] = v;
         bv = v;
         bi = c;
       }
@@ -474,17 +499,18 @@ __global__ void __launch_bounds__(256) perm_update(Ws ws) {
           }
         }
       } else {
-        for (int64_t b = lane; b < ws.k; b += 32) {
-          const int pb = ws.pos[b];
-          const int g2 = pb >> 2;
-          long long v;
-          if (g2 == ga || g2 == gb)
-            v = ua + ws.u[b] + ws.part[((g2 == ga ? 0 : 4) + (pb & 3)) * ws.k + a];
-          else
-            v = ws.gain[a * ws.k + b];
-          if (v > bv || (v == bv && static_cast<int>(b) < bi)) {
-            bv = v;
-            bi = static_cast<int>(b);
+        // the 8 new entries are in `row` now; scan it two entries at a time
+        __syncwarp();
+        const longlong2* row2 = reinterpret_cast<const longlong2*>(row);
+        for (int64_t h = lane; h < ws.k / 2; h += 32) {
+          const longlong2 v = row2[h];
+          if (v.x > bv || (v.x == bv && static_cast<int>(2 * h) < bi)) {
+            bv = v.x;
+            bi = static_cast<int>(2 * h);
+          }
+          if (v.y > bv || (v.y == bv && static_cast<int>(2 * h + 1) < bi)) {
+            bv = v.y;
+            bi = static_cast<int>(2 * h + 1);
           }
         }
       }
@@ -495,6 +521,7 @@ __global__ void __launch_bounds__(256) perm_update(Ws ws) {
       ws.best_idx[a] = bi;
     }
   }
+  pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------- column gather
@@ -531,7 +558,7 @@ inline Layout layout(int64_t n, int64_t k) {
   l.tc = o;        o += up256(4 * 16 * static_cast<size_t>(n));
   l.gain = o;      o += up256(8 * static_cast<size_t>(k) * static_cast<size_t>(k));
   l.u = o;         o += up256(8 * static_cast<size_t>(k));
-  l.part = o;      o += up256(8 * 8 * static_cast<size_t>(k));
+  l.part = o;      o += up256(2 * 8 * 8 * static_cast<size_t>(k));
   l.best_val = o;  o += up256(8 * static_cast<size_t>(k));
   l.best_idx = o;  o += up256(4 * static_cast<size_t>(k));
   l.pos = o;       o += up256(4 * static_cast<size_t>(k));
@@ -541,10 +568,10 @@ inline Layout layout(int64_t n, int64_t k) {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Rows per slice so that `blocks` x slices covers about two waves, slices of
+// Rows per slice so that `blocks` x slices covers about `waves` waves, slices of
 // at least `min_rows` rows, a multiple of kRowChunk.
-inline int64_t slice_rows(int64_t n, int64_t blocks, int64_t min_rows) {
-  const int64_t want = 2 * static_cast<int64_t>(sm_count());
+inline int64_t slice_rows(int64_t n, int64_t blocks, int64_t min_rows, int waves = 2) {
+  const int64_t want = waves * static_cast<int64_t>(sm_count());
   int64_t slices = blocks >= want ? 1 : ceil_div(want, blocks);
   slices = std::min(slices, std::max<int64_t>(1, ceil_div(n, min_rows)));
   const int64_t rows = ceil_div(ceil_div(n, slices), kRowChunk) * kRowChunk;
@@ -598,6 +625,7 @@ sp24_status sp24_permute_search(const void* W, int64_t N, int64_t K, const doubl
 
   cudaError_t e = cudaMemsetAsync(ws.st, 0, sizeof(State), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(ws.u, 0, 8 * static_cast<size_t>(K), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws.part, 0, 2 * 8 * 8 * static_cast<size_t>(K), s);
   if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync", e);
 
   const unsigned ex = static_cast<unsigned>(std::min<int64_t>(ceil_div(K, 256), 8));
@@ -627,7 +655,7 @@ sp24_status sp24_permute_search(const void* W, int64_t N, int64_t K, const doubl
   SP24_TRY(launch_kernel(perm_rowbest_full, dim3(wrows), dim3(256), 0, s, 1, ws));
 
   const int64_t pcols = ceil_div(K, 256);
-  const int64_t prows = slice_rows(N, pcols, 64);
+  const int64_t prows = slice_rows(N, pcols, 64, 4);
   const dim3 pgrid(static_cast<unsigned>(pcols), static_cast<unsigned>(ceil_div(N, prows)));
   const unsigned fx = static_cast<unsigned>(std::min<int64_t>(ceil_div(N, 256), 64));
   if (max_swaps > (INT64_MAX >> 1)) max_swaps = INT64_MAX >> 1;
