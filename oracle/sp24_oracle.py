@@ -507,3 +507,50 @@ def best_kept_score_bruteforce(q: np.ndarray, n_keep: int) -> int:
 def permute_columns(a: np.ndarray, perm: np.ndarray) -> np.ndarray:
     """A[:, perm]: column j of the result is column perm[j] of A."""
     return np.asarray(a)[:, np.asarray(perm)]
+
+
+# ---------------------------------------------------------------------------
+# f3  3x3 convolution as a GEMM with 2:4 along (kh, kw, Cin)
+#     [Orin ch.7] 2.2 A.3 (large 3x3 convolutions, large batch or high
+#     resolution, are good candidates) and 2.1 (groups of 4 along the input
+#     channels)
+# ---------------------------------------------------------------------------
+# Readings: stride 1, zero padding 1, NHWC activations X[n][h][w][c], weights
+# W[co][kh][kw][c].  The GEMM view has M = n*H*W output pixels, N = Cout and
+# K = 9*Cin ordered (kh, kw, c), so a group of 4 runs along Cin inside one tap
+# when Cin % 4 == 0; pruning and compression act on W viewed as [Cout][9*Cin].
+def conv3x3_nhwc(x: np.ndarray, w4: np.ndarray) -> np.ndarray:
+    """y[n,h,w,co] = sum_{kh,kw,c} x[n, h+kh-1, w+kw-1, c] * w4[co,kh,kw,c],
+    x zero outside the image; float64.  One matmul per tap."""
+    x = np.asarray(x, dtype=np.float64)
+    w4 = np.asarray(w4, dtype=np.float64)
+    n, hh, ww, c = x.shape
+    co = w4.shape[0]
+    xp = np.zeros((n, hh + 2, ww + 2, c))
+    xp[:, 1:hh + 1, 1:ww + 1, :] = x
+    y = np.zeros((n, hh, ww, co))
+    for kh in range(3):
+        for kw in range(3):
+            y += xp[:, kh:kh + hh, kw:kw + ww, :] @ w4[:, kh, kw, :].T
+    return y
+
+
+def conv3x3_weight_as_gemm(w4: np.ndarray) -> np.ndarray:
+    """W[co][kh][kw][c] -> [Cout][9*Cin], column (kh*3 + kw)*Cin + c."""
+    w4 = np.asarray(w4)
+    return w4.reshape(w4.shape[0], -1)
+
+
+def im2col3x3(x: np.ndarray) -> np.ndarray:
+    """A[(n*H + h)*W + w][(kh*3 + kw)*Cin + c] = x[n, h+kh-1, w+kw-1, c]
+    (0 outside the image): the GEMM operand of conv3x3_nhwc."""
+    x = np.asarray(x)
+    n, hh, ww, c = x.shape
+    a = np.zeros((n, hh, ww, 9, c), dtype=x.dtype)
+    for kh in range(3):
+        for kw in range(3):
+            dh, dw = kh - 1, kw - 1
+            h0, h1 = max(0, -dh), min(hh, hh - dh)
+            w0, w1 = max(0, -dw), min(ww, ww - dw)
+            a[:, h0:h1, w0:w1, kh * 3 + kw, :] = x[:, h0 + dh:h1 + dh, w0 + dw:w1 + dw, :]
+    return a.reshape(n * hh * ww, 9 * c)

@@ -544,3 +544,81 @@ def test_perm_columns_leave_the_product_unchanged():
     xp, wp = O.permute_columns(x, perm), O.permute_columns(w, perm)
     assert (xp @ wp.T == x @ w.T).all()
     assert (xp[:, np.argsort(perm)] == x).all()
+
+
+# ------------------------------------------------- 3x3 convolution as a GEMM
+# [Orin ch.7] 2.2 A.3 and 2.1: stride 1, zero padding 1, NHWC, groups of 4
+# along (kh, kw, Cin).
+
+def _conv3x3_loops(x, w4):
+    """Seven nested loops over integers, bounds checked per term."""
+    n, hh, ww, c = x.shape
+    co = w4.shape[0]
+    y = [[[[0] * co for _ in range(ww)] for _ in range(hh)] for _ in range(n)]
+    for b in range(n):
+        for h in range(hh):
+            for w in range(ww):
+                for o in range(co):
+                    s = 0
+                    for kh in range(3):
+                        for kw in range(3):
+                            ih, iw = h + kh - 1, w + kw - 1
+                            if 0 <= ih < hh and 0 <= iw < ww:
+                                for ci in range(c):
+                                    s += int(x[b, ih, iw, ci]) * int(w4[o, kh, kw, ci])
+                    y[b][h][w][o] = s
+    return np.array(y, dtype=np.float64)
+
+
+def test_conv3x3_equals_bruteforce_and_im2col_gemm():
+    rng = np.random.default_rng(31)
+    x = rng.integers(-4, 5, size=(2, 4, 5, 8))
+    w4 = rng.integers(-4, 5, size=(3, 3, 3, 8))
+    want = _conv3x3_loops(x, w4)
+    assert np.array_equal(O.conv3x3_nhwc(x, w4), want)
+    a = O.im2col3x3(x)
+    assert a.shape == (2 * 4 * 5, 72)
+    assert np.array_equal((a @ O.conv3x3_weight_as_gemm(w4).T).reshape(want.shape), want)
+
+
+def test_conv3x3_special_kernels():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((1, 4, 3, 4))
+    # centre tap only: a 1x1 convolution
+    w4 = np.zeros((5, 3, 3, 4))
+    w4[:, 1, 1, :] = rng.standard_normal((5, 4))
+    assert np.allclose(O.conv3x3_nhwc(x, w4), x @ w4[:, 1, 1, :].T, rtol=0, atol=1e-15)
+    # top-left tap with the identity over channels: y[h][w] = x[h-1][w-1]
+    w4 = np.zeros((4, 3, 3, 4))
+    w4[:, 0, 0, :] = np.eye(4)
+    y = O.conv3x3_nhwc(x, w4)
+    assert (y[:, 0, :, :] == 0).all() and (y[:, :, 0, :] == 0).all()
+    assert np.array_equal(y[:, 1:, 1:, :], x[:, :-1, :-1, :])
+
+
+def test_im2col_columns_follow_taps_then_channels():
+    x = np.arange(1, 1 + 2 * 2 * 8).reshape(1, 2, 2, 8)
+    a = O.im2col3x3(x)
+    # pixel (0, 0): taps with kh = 0 or kw = 0 read outside the image
+    assert (a[0, :8 * 4] == 0).all()              # taps (0,0) (0,1) (0,2) (1,0)
+    assert (a[0, 4 * 8:5 * 8] == x[0, 0, 0]).all()  # tap (1,1) = the pixel itself
+    assert (a[0, 5 * 8:6 * 8] == x[0, 0, 1]).all()  # tap (1,2) = right neighbour
+    assert (a[0, 8 * 8:9 * 8] == x[0, 1, 1]).all()  # tap (2,2) = down-right
+    # pixel (1, 1) (row 3): tap (0,0) = x[0,0]
+    assert (a[3, 0:8] == x[0, 0, 0]).all()
+
+
+def test_sparse_conv3x3_groups_stay_inside_one_tap():
+    rng = np.random.default_rng(33)
+    x = rng.integers(-3, 4, size=(1, 3, 4, 8))
+    w4 = rng.integers(-3, 4, size=(4, 3, 3, 8)).astype(np.float64)
+    wg = O.conv3x3_weight_as_gemm(w4)
+    keep = O.prune(wg, O.MAGNITUDE, 2)
+    # with Cin % 4 == 0 every group of 4 columns lies in one (kh, kw) tap
+    for g in range(wg.shape[1] // 4):
+        assert len({(4 * g + i) // 8 for i in range(4)}) == 1
+    w4m = np.where(keep, wg, 0.0).reshape(w4.shape)
+    want = _conv3x3_loops(x, w4m.astype(np.int64))
+    vals, meta = O.compress(wg, keep)
+    got, _ = O.gemm(O.im2col3x3(x).astype(np.float64), vals, meta, wg.shape[1])
+    assert np.array_equal(got.reshape(want.shape), want)
