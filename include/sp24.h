@@ -307,6 +307,25 @@ typedef struct sp24_gemm_plan_t {
 
 sp24_status sp24_gemm_plan(int64_t M, int64_t N, int64_t K, int dtype, sp24_gemm_plan_t* plan);
 
+/* ------------------------------------------------------ 3x3 convolution */
+
+/* 3x3 convolution input as the token operand of sp24_gemm ([Orin ch.7]
+ * 2.2 A.3: large 3x3 convolutions at large batch or high resolution are good
+ * 2:4 candidates; 2.1: groups of 4 run along the input channels).  Stride 1,
+ * zero padding 1, NHWC:
+ *   A[(b*H + h)*W + w][(kh*3 + kw)*C + c] = X[b][h+kh-1][w+kw-1][c], or 0
+ *   when (h+kh-1, w+kw-1) lies outside the H x W image.
+ * sp24_gemm(A, M = B*H*W, K = 9*C, ...) with the weights W[Cout][3][3][C]
+ * pruned and compressed as the [Cout][9*C] matrix then gives the convolution
+ * output Y[B*H*W][Cout] (NHWC); with C % 4 == 0 every group of 4 lies inside
+ * one (kh, kw) tap.  For INT8, quantise X first (elem_bytes 1): a padded 0 is
+ * the int8 code 0.
+ *   X: [B][H][W][C] elements of elem_bytes bytes (2: bf16, 1: int8).
+ *   A: [B*H*W][9*C] elements of the same size (written).
+ * Rules: B, H, W, C >= 0; elem_bytes in {1, 2}; C * elem_bytes % 16 == 0. */
+sp24_status sp24_im2col3x3(const void* X, int64_t B, int64_t H, int64_t W, int64_t C,
+                           int elem_bytes, void* A, void* stream);
+
 /* ------------------------------------------------- allocation-free variant */
 
 /* Largest K accepted by sp24_prune_wanda_noalloc. */

@@ -4,3 +4,4 @@
 #include "prune.cu"
 #include "gemm_sp.cu"
 #include "permute.cu"
+#include "conv.cu"

@@ -122,3 +122,20 @@ def permute_columns(A: torch.Tensor, perm: torch.Tensor) -> torch.Tensor:
     out = torch.empty_like(A)
     _b.sp24_permute_columns(A, perm, out)
     return out
+
+
+def im2col3x3(X: torch.Tensor) -> torch.Tensor:
+    """NHWC X [B, H, W, C] -> the 3x3 convolution's GEMM operand [B*H*W, 9*C]."""
+    Bn, H, W, C = X.shape
+    A = torch.empty((Bn * H * W, 9 * C), dtype=X.dtype, device=X.device)
+    _b.sp24_im2col3x3(X, A)
+    return A
+
+
+def conv3x3(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, Cout: int,
+            **gemm_kwargs) -> torch.Tensor:
+    """3x3 convolution (stride 1, padding 1) of NHWC X with 2:4 weights
+    compressed from W[Cout][3][3][C] viewed as [Cout][9*C].  Returns NHWC Y."""
+    Bn, H, W, _ = X.shape
+    y = gemm(im2col3x3(X), vals, meta, Cout, **gemm_kwargs)
+    return y.view(Bn, H, W, Cout)

@@ -73,6 +73,7 @@ SIGNATURES = {
     "sp24_permute_search": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_int, _c_i64, _c_p, _c_p,
                                      _c_size, _c_p, _c_p]),
     "sp24_permute_columns": (_c_int, [_c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p]),
+    "sp24_im2col3x3": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_int, _c_p, _c_p]),
 }
 
 
@@ -282,6 +283,13 @@ def sp24_permute_columns(A: torch.Tensor, perm: torch.Tensor, A_out: torch.Tenso
     rows, K = A.shape
     _check(lib().sp24_permute_columns(_ptr(A), rows, K, A.element_size(), _ptr(perm),
                                       _ptr(A_out), _stream(stream)), "sp24_permute_columns")
+
+
+def sp24_im2col3x3(X: torch.Tensor, A: torch.Tensor, stream=None) -> None:
+    """X NHWC [B][H][W][C] -> A [B*H*W][9*C] (3x3, stride 1, zero padding 1)."""
+    Bn, H, W, C = X.shape
+    _check(lib().sp24_im2col3x3(_ptr(X), Bn, H, W, C, X.element_size(), _ptr(A),
+                                _stream(stream)), "sp24_im2col3x3")
 
 
 def sp24_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -177,3 +177,14 @@ def test_permute_host_validation(lib):
     assert g(FAKE, 0, 16, 2, FAKE, FAKE + 256, None) == B.SP24_OK           # nothing to do
     assert g(FAKE + 4, 4, 16, 2, FAKE, FAKE + 256, None) == B.SP24_ERR_ALIGN
     assert lib.sp24_strerror(B.SP24_ERR_INDEX).decode().startswith("a permutation entry")
+
+
+def test_im2col_host_validation(lib):
+    f = lib.sp24_im2col3x3
+    assert f(FAKE, 1, 4, 4, 8, 3, FAKE, None) == B.SP24_ERR_ARG      # element size
+    assert f(FAKE, -1, 4, 4, 8, 2, FAKE, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 0, 4, 4, 8, 2, FAKE, None) == B.SP24_OK          # nothing to do
+    assert f(None, 1, 4, 4, 8, 2, FAKE, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 1, 4, 4, 12, 2, FAKE, None) == B.SP24_ERR_ALIGN  # 24-byte pixels
+    assert f(FAKE, 1, 4, 4, 8, 1, FAKE, None) == B.SP24_ERR_ALIGN   # 8-byte pixels
+    assert f(FAKE + 8, 1, 4, 4, 8, 2, FAKE, None) == B.SP24_ERR_ALIGN
