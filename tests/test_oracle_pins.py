@@ -313,6 +313,49 @@ def test_nearest_rank_quantile_vs_numpy():
     assert O.quantile_abs(v[:10000], 0.9999) == 9999.0
 
 
+def test_tensor_scale_hand_cases():
+    # [Ampere-sparsity] "PTQ and QAT": the activation scale covers 99.99 % of
+    # the values.  |v| = 1 .. 10001 (signs mixed, order shuffled): the nearest
+    # rank is ceil(0.9999 * 10001) = 10000, so t = 10000 and s = 10000 / 127
+    # in float32 whatever the signs or the order.
+    rng = np.random.default_rng(12)
+    mag = np.arange(1, 10002, dtype=np.float64)
+    v = rng.permutation(mag * np.where(rng.random(10001) < 0.5, -1.0, 1.0))
+    expect = np.float32(np.float32(10000.0) / np.float32(127.0))
+    assert O.tensor_scale(v) == expect
+    assert O.tensor_scale(v, 0.9999) == expect          # the default coverage is 0.9999
+    assert O.tensor_scale(v.reshape(1, -1)) == expect   # layout does not matter
+    # all-zero tensor: the quantile is 0 and the scale is 1
+    assert O.tensor_scale(np.zeros((3, 5))) == np.float32(1.0)
+    assert O.tensor_scale(-np.zeros(7)) == np.float32(1.0)
+
+
+def test_tensor_scale_ranks_over_every_entry_of_a_matrix():
+    # A [3, 6667] matrix of 20001 distinct magnitudes.  The rank over all
+    # entries is ceil(0.9999 * 20001) = 19999: the third largest magnitude.
+    # Every row (6667 entries, rank 6667) and every column (3 entries, rank 3)
+    # takes its own maximum under the same rule, and the fixture places the
+    # three largest so that none of those equals the third largest: the
+    # largest at (1, 5), the second at (0, 9), the third at (0, 5).
+    rows, cols = 3, 6667
+    rng = np.random.default_rng(13)
+    mags = rng.permutation(np.arange(1, rows * cols - 2, dtype=np.float64))
+    x = np.empty((rows, cols))
+    slots = [(r, c) for r in range(rows) for c in range(cols)
+             if (r, c) not in ((1, 5), (0, 9), (0, 5))]
+    for (r, c), m in zip(slots, mags):
+        x[r, c] = m
+    top = float(rows * cols)
+    x[1, 5], x[0, 9], x[0, 5] = top, top - 1, top - 2
+    x = x * np.where(rng.random(x.shape) < 0.5, -1.0, 1.0)
+    assert O.nearest_rank(0.9999, rows * cols) == rows * cols - 2
+    third = np.float32(np.float32(top - 2) / np.float32(127.0))
+    assert O.tensor_scale(x) == third
+    per_row = {O.tensor_scale(x[r]) for r in range(rows)}
+    per_col = {O.tensor_scale(x[:, c]) for c in range(cols)}
+    assert third not in per_row and third not in per_col
+
+
 def test_zero_row_scale_is_one():
     assert O.scale_from_quantile(0.0) == np.float32(1.0)
     w = np.zeros((1, 8))
