@@ -344,8 +344,9 @@ sp24_status sp24_im2col3x3(const void* X, int64_t B, int64_t H, int64_t W, int64
  *     that loads the library keeps it until the process exits.  K larger than
  *     SP24_NOALLOC_MAX_K returns SP24_ERR_UNSUPPORTED before any launch.
  *   - The first call on a device looks up the array's device address (a
- *     one-time set-up per device); make that first call before any stream
- *     capture on the device.
+ *     one-time set-up per device, repeated only if the device's context has
+ *     changed since, e.g. after cudaDeviceReset); make that first call before
+ *     any stream capture on the device.
  *   - All calls share the one array and each call overwrites all K entries it
  *     uses before reading them.  Calls that overlap on the GPU (for example on
  *     two streams at once) race on it and must be serialised by the caller.

@@ -11,6 +11,8 @@
 // [Ampere-sparsity] NVIDIA x Tencent article, Figure 1 (values + index
 // metadata), Figure 4 (progressive 25 % -> 50 %), "PTQ and QAT" (99.99 %
 // coverage scale).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "sp24_device.cuh"
@@ -1077,25 +1079,59 @@ __device__ __align__(256) double g_noalloc_norms[SP24_NOALLOC_MAX_K];
 
 namespace {
 constexpr int kNoallocMaxDevices = 64;
-double* g_noalloc_ptr[kNoallocMaxDevices];   // device address of the array, per device
+
+// The array's device address on one device, and the context it was looked up
+// in.  A module's globals move when its context is destroyed and recreated
+// (cudaDeviceReset, for instance), so the address is looked up again whenever
+// the device's current context differs from the one recorded here.
+struct NoallocSlot {
+  CUcontext ctx;
+  double* ptr;
+};
+NoallocSlot g_noalloc_slot[kNoallocMaxDevices];
 std::mutex g_noalloc_mu;
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+CUcontext current_ctx() {
+  CUcontext c = nullptr;
+  const CtxGetCurrentFn f = ctx_get_current();
+  if (f == nullptr || f(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
+}
+
 // Device address of g_noalloc_norms on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached.
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress, with the device current, on the first call and after
+// any change of the device's context, and cached otherwise.
 sp24_status noalloc_norms(double** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
   if (dev < 0 || dev >= kNoallocMaxDevices) return SP24_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  const CUcontext before = current_ctx();
+  if (slot.ptr == nullptr || before == nullptr || before != slot.ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_norms);
     if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress", e);
-    g_noalloc_ptr[dev] = static_cast<double*>(p);
+    slot.ptr = static_cast<double*>(p);
+    slot.ctx = current_ctx();   // the lookup creates the primary context if needed
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return SP24_OK;
 }
 }  // namespace

@@ -62,6 +62,31 @@ def test_no_alloc_matches_workspace_prune_on_consecutive_calls():
     assert torch.equal(got3, ref3)
 
 
+def test_no_alloc_separate_norm_kernel_on_consecutive_calls():
+    # Row tiles x calibration rows above 8192 make the library compute the
+    # column norms with their own kernel, which writes them to the scratch
+    # array, and the prune kernel then reads them back from it (the fused
+    # path above keeps them on chip).  Call 1: 11008 rows (86 row tiles) x
+    # 128 calibration rows.  Call 2: 1024 rows (8 row tiles) x 1100
+    # calibration rows, smaller K, with a mask_in: norms left over from call 1
+    # in the shared array would change its mask.
+    Wa = I.normal_bf16((11008, 512), 0.02, seed=81).cuda()
+    Xa = I.normal_bf16((128, 512), 1.0, seed=82).cuda()
+    Wb = I.normal_bf16((1024, 264), 0.02, seed=83).cuda()
+    Xb = I.normal_bf16((1100, 264), 1.0, seed=84).cuda()
+    got_a = _no_alloc(Wa, Xa, 3)
+    mb = _with_workspace(Wb, Xb, 3)
+    got_b = _no_alloc(Wb, Xb, 2, mb)
+    ref_a = _with_workspace(Wa, Xa, 3)
+    ref_b = _with_workspace(Wb, Xb, 2, mb)
+    # call 3 repeats call 1 after call 2 left other norms in the array
+    got_a2 = _no_alloc(Wa, Xa, 3)
+    assert B.sp24_device_status() == B.SP24_OK
+    assert torch.equal(got_a, ref_a)
+    assert torch.equal(got_b, ref_b)
+    assert torch.equal(got_a2, ref_a)
+
+
 def test_no_alloc_rejects_k_above_limit():
     big = B.SP24_NOALLOC_MAX_K + 8
     W = torch.empty((1, big), dtype=torch.bfloat16, device="cuda")
