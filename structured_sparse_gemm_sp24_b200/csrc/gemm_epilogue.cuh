@@ -66,20 +66,35 @@ __device__ __forceinline__ float epi_value(uint32_t acc, float cscale) {
 // lane/8 for stmatrix; the box row is 64 bytes and its 16-byte chunk index is
 // XORed with bits 1-2 of the row (64-byte swizzle).
 template <int kDtype, int NB>
-__device__ __forceinline__ void stage_vec(const uint32_t (&r)[32], uint32_t stg, int lane,
-                                          const float (&cs)[4]) {
+__device__ __forceinline__ void pack_vec(const uint32_t (&r)[32], const float (&cs)[4],
+                                         uint32_t (&pk)[16]) {
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    uint32_t p[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int i = 16 * (q >> 1) + 4 * b + 2 * (q & 1);
-      p[q] = pack_bf16x2(epi_value<kDtype>(r[i], cs[q]), epi_value<kDtype>(r[i + 1], cs[q]));
+      pk[4 * b + q] = pack_bf16x2(epi_value<kDtype>(r[i], cs[q]), epi_value<kDtype>(r[i + 1], cs[q]));
     }
+  }
+}
+
+template <int NB>
+__device__ __forceinline__ void stmatrix_vec(const uint32_t (&pk)[16], uint32_t stg, int lane) {
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
     const int tok = 8 * b + (lane & 7);
     const int chunk = (lane >> 3) ^ ((tok >> 1) & 3);
-    stmatrix_x4_trans(stg + tok * 64 + chunk * 16, p[0], p[1], p[2], p[3]);
+    stmatrix_x4_trans(stg + tok * 64 + chunk * 16, pk[4 * b], pk[4 * b + 1], pk[4 * b + 2],
+                      pk[4 * b + 3]);
   }
+}
+
+template <int kDtype, int NB>
+__device__ __forceinline__ void stage_vec(const uint32_t (&r)[32], uint32_t stg, int lane,
+                                          const float (&cs)[4]) {
+  uint32_t pk[16];
+  pack_vec<kDtype, NB>(r, cs, pk);
+  stmatrix_vec<NB>(pk, stg, lane);
 }
 
 // One-channel-per-thread path (thread `lane` owns channel c0 + lane), NT tokens.
@@ -124,12 +139,44 @@ __device__ __forceinline__ void epi_load(const EpiWarp& e, int chunk, bool half,
   }
 }
 
+// Stages one loaded chunk (c) of this warp and issues its TMA store.
+template <int kDtype, int OUTK>
+__device__ __forceinline__ void epi_store_chunk(const EpiWarp& e, const CUtensorMap* tmap_y,
+                                                const CUtensorMap* tmap_y16, int c, bool half,
+                                                int lane, const uint32_t (&r)[32]) {
+  const int64_t t0 = e.tok0 + c * kEpiChunk;
+  if (e.c0 >= e.n || t0 >= e.m) return;   // no channel of this quadrant / token of the chunk
+  if (lane == 0) bulk_wait_read<0>();     // this warp's previous store read out
+  __syncwarp();
+  if (e.vec) {
+    if (half) stage_vec<kDtype, 2>(r, smem_u32(e.stg), lane, e.cs);
+    else stage_vec<kDtype, 4>(r, smem_u32(e.stg), lane, e.cs);
+  } else if (e.c0 + lane < e.n) {
+    if (half) stage_scalar<kDtype, OUTK, 16>(r, e.stg, lane, e.cbox, e.cs[0], e.sy);
+    else stage_scalar<kDtype, OUTK, 32>(r, e.stg, lane, e.cbox, e.cs[0], e.sy);
+  }
+  fence_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(half ? tmap_y16 : tmap_y, e.stg, e.c0, static_cast<int32_t>(t0));
+    bulk_commit();
+  }
+}
+
 // Drains this warp's chunks (grp, grp + 2, ...) of one tile.  With BN % 32 ==
 // 16 the tile's last chunk holds 16 tokens and is stored through `tmap_y16`
 // (16-token boxes), so no store reaches past the tile.  `release` runs once
 // the warp's last tensor-memory load has completed (the accumulator may then
 // be reused); all lanes call it.
-template <int kDtype, int OUTK, int BN, class Release>
+//   kHoldAll = false: the next chunk's load is issued before the current
+//     chunk is staged (two chunks of registers); the accumulator is released
+//     after the last load, i.e. after most of the staging.  Used where a
+//     second accumulator lets the next tile's MMAs run meanwhile.
+//   kHoldAll = true (bf16 output through the transposing path; otherwise as
+//     false): all of the warp's chunks are loaded and packed to bf16 pairs in
+//     registers first and the accumulator is released before any staging, so
+//     with a single accumulator the next tile's MMAs wait only for the loads.
+template <int kDtype, int OUTK, int BN, bool kHoldAll, class Release>
 __device__ __forceinline__ void epilogue_tile(const EpiWarp& e, const CUtensorMap* tmap_y,
                                               const CUtensorMap* tmap_y16, int grp, int lane,
                                               Release&& release) {
@@ -139,34 +186,59 @@ __device__ __forceinline__ void epilogue_tile(const EpiWarp& e, const CUtensorMa
   static_assert(kChunks >= 2, "each warp of a quadrant must own a chunk of every tile");
   constexpr int kMaxMine = (kChunks + 1) / 2;
   const int nmine = (kChunks - grp + 1) / 2;
-  const bool live = e.c0 < e.n;   // some channel of this quadrant exists
-  uint32_t r[2][32];
-  if (nmine > 0) epi_load(e, grp, kHalfTail && grp == kChunks - 1, r[0]);
+  if (kHoldAll && OUTK == SP24_OUT_BF16 && e.vec) {
+    // two chunks at a time: load, wait, pack to bf16 pairs (16 registers a
+    // chunk); the accumulator is released once every chunk is packed
+    uint32_t pk[kMaxMine][16];
 #pragma unroll
-  for (int i = 0; i < kMaxMine; ++i) {
-    if (i < nmine) {
+    for (int i = 0; i < kMaxMine; i += 2) {
+      uint32_t r[2][32];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = grp + 2 * (i + u);
+        if (i + u < kMaxMine && i + u < nmine) epi_load(e, c, kHalfTail && c == kChunks - 1, r[u]);
+      }
+      tmem_ld_wait();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = grp + 2 * (i + u);
+        if (i + u < kMaxMine && i + u < nmine) {
+          if (kHalfTail && c == kChunks - 1) pack_vec<kDtype, 2>(r[u], e.cs, pk[i + u]);
+          else pack_vec<kDtype, 4>(r[u], e.cs, pk[i + u]);
+        }
+      }
+    }
+    release();
+#pragma unroll
+    for (int i = 0; i < kMaxMine; ++i) {
       const int c = grp + 2 * i;
       const bool half = kHalfTail && c == kChunks - 1;
-      tmem_ld_wait();   // chunk i landed (and nothing else is outstanding)
-      if (i + 1 < nmine) epi_load(e, c + 2, kHalfTail && c + 2 == kChunks - 1, r[(i + 1) & 1]);
-      else release();
       const int64_t t0 = e.tok0 + c * kEpiChunk;
-      if (live && t0 < e.m) {
-        if (lane == 0) bulk_wait_read<0>();         // this warp's previous store read out
+      if (i < nmine && e.c0 < e.n && t0 < e.m) {
+        if (lane == 0) bulk_wait_read<0>();     // this warp's previous store read out
         __syncwarp();
-        if (e.vec) {
-          if (half) stage_vec<kDtype, 2>(r[i & 1], smem_u32(e.stg), lane, e.cs);
-          else stage_vec<kDtype, 4>(r[i & 1], smem_u32(e.stg), lane, e.cs);
-        } else if (e.c0 + lane < e.n) {
-          if (half) stage_scalar<kDtype, OUTK, 16>(r[i & 1], e.stg, lane, e.cbox, e.cs[0], e.sy);
-          else stage_scalar<kDtype, OUTK, 32>(r[i & 1], e.stg, lane, e.cbox, e.cs[0], e.sy);
-        }
+        if (half) stmatrix_vec<2>(pk[i], smem_u32(e.stg), lane);
+        else stmatrix_vec<4>(pk[i], smem_u32(e.stg), lane);
         fence_async_shared();
         __syncwarp();
         if (lane == 0) {
           tma_store_2d(half ? tmap_y16 : tmap_y, e.stg, e.c0, static_cast<int32_t>(t0));
           bulk_commit();
         }
+      }
+    }
+  } else {
+    uint32_t r[2][32];
+    if (nmine > 0) epi_load(e, grp, kHalfTail && grp == kChunks - 1, r[0]);
+#pragma unroll
+    for (int i = 0; i < kMaxMine; ++i) {
+      if (i < nmine) {
+        const int c = grp + 2 * i;
+        tmem_ld_wait();   // chunk i landed (and nothing else is outstanding)
+        if (i + 1 < nmine) epi_load(e, c + 2, kHalfTail && c + 2 == kChunks - 1, r[(i + 1) & 1]);
+        else release();
+        epi_store_chunk<kDtype, OUTK>(e, tmap_y, tmap_y16, c, kHalfTail && c == kChunks - 1, lane,
+                                      r[i & 1]);
       }
     }
   }

@@ -213,7 +213,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
       epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
       e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       e.tok0 = static_cast<int64_t>(tt) * BN;
-      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, &tmap_y16, grp, lane, [&] {
+      epilogue_tile<kDtype, OUTK, BN, (ACC == 1)>(e, &tmap_y, &tmap_y16, grp, lane, [&] {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(map_peer(smem_u32(&tempty_bar[acc]), 0));
@@ -280,6 +280,7 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
   const int64_t row_tile_bytes = 256 * (g.k / 2) * el;
   int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = group_rows_override(gr);
   gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
   a.group_rows = static_cast<int>(gr);
   a.y_box = y_box;

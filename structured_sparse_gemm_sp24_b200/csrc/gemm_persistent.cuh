@@ -56,6 +56,15 @@ struct PersistArgs {
   int y_box;         // channels per epilogue store box: min(32, N)
 };
 
+// SP24_GEMM_GROUP_ROWS = n > 0: raster group height in weight row tiles
+// (tuning override of the persistent kernels; results do not depend on it).
+inline int64_t group_rows_override(int64_t gr) {
+  const char* e = std::getenv("SP24_GEMM_GROUP_ROWS");
+  if (!e) return gr;
+  const long v = std::atol(e);
+  return v > 0 ? static_cast<int64_t>(v) : gr;
+}
+
 // Linear tile index -> (row tile, token tile) in the grouped order.
 __device__ __forceinline__ void tile_coords(int t, const PersistArgs& a, int& rt, int& tt) {
   const int per_group = a.group_rows * a.tok_tiles;
@@ -216,7 +225,7 @@ gemm_sp_persistent(const __grid_constant__ CUtensorMap tmap_a,
       epi_scales<kDtype, OUTK>(e, lane, args.s_w, sx);
       e.tmem = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * BN;
       e.tok0 = static_cast<int64_t>(tt) * BN;
-      epilogue_tile<kDtype, OUTK, BN>(e, &tmap_y, &tmap_y, grp, lane, [&] {
+      epilogue_tile<kDtype, OUTK, BN, false>(e, &tmap_y, &tmap_y, grp, lane, [&] {
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty_bar[acc]);   // accumulator drained
@@ -262,6 +271,7 @@ sp24_status launch_persistent(const CUtensorMap& ma, const CUtensorMap& mb, cons
   // raster group: as many weight row tiles as fit ~24 MB of compressed weights
   const int64_t row_tile_bytes = 128 * (g.k / 2) * (kDtype == SP24_BF16 ? 2 : 1);
   int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  gr = group_rows_override(gr);
   gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
   a.group_rows = static_cast<int>(gr);
   a.y_box = y_box;
