@@ -1,5 +1,7 @@
 """Host-side pieces of bench.py that need no GPU: the ncu traffic table it
-reads for the roofline and the source hash that invalidates it."""
+reads for the roofline, the source hash that invalidates it, the peak
+denominators and the bounded CPU-oracle sample."""
+import json
 import os
 
 import bench
@@ -8,31 +10,66 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _rows():
-    with open(os.path.join(ROOT, "profiles", "gemm_dram_traffic.md")) as f:
-        for line in f:
-            cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) == 5 and cells[3].isdigit():
-                yield cells
+    with open(os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")) as f:
+        return json.load(f)["rows"]
 
 
-def test_traffic_table_parses_and_covers_default_workload():
-    rows = list(_rows())
+def test_traffic_table_parses():
+    rows = _rows()
     assert rows, "no data rows"
-    names = {r[0] for r in rows}
-    assert "bert_fc1_wanda_3072x768_m4096" in names
-    for wl, plan, kernel, traffic, h in rows:
-        assert int(traffic) > 0 and kernel.startswith("gemm_sp") and len(h) == 16
-        assert bench.family_of(plan) in bench.FAMILY_SOURCES
+    for r in rows:
+        assert int(r["traffic_bytes"]) > 0 and r["kernel"].startswith("gemm_sp")
+        assert len(r["family_src_hash"]) == 16
+        assert bench.family_of(r["plan"]) in bench.FAMILY_SOURCES
 
 
-def test_traffic_lookup_follows_plan_and_source_hash():
-    for wl, plan, _, traffic, h in _rows():
-        cur = bench.gemm_src_hash(bench.family_of(plan))
+def test_traffic_lookup_follows_plan_and_source_hash(tmp_path):
+    for r in _rows():
+        cur = bench.gemm_src_hash(bench.family_of(r["plan"]))
         assert len(cur) == 16
-        assert bench.gemm_traffic(wl, plan) == (int(traffic) if h == cur else None)
-        other = "single" if plan.startswith("pair") else "pair256"
-        assert bench.gemm_traffic(wl, other) is None   # another kernel: no number
+        want = int(r["traffic_bytes"]) if r["family_src_hash"] == cur else None
+        assert bench.gemm_traffic(r["workload"], r["plan"]) == want
+        other = "single" if r["plan"].startswith("pair") else "pair256"
+        assert bench.gemm_traffic(r["workload"], other) is None   # another kernel: no number
     assert bench.gemm_traffic("no_such_workload", "pair256") is None
+    # a row recorded with the current hash is found; a stale hash is not
+    cur = bench.gemm_src_hash("pair")
+    p = tmp_path / "t.json"
+    p.write_text(json.dumps({"rows": [
+        {"workload": "w", "plan": "pair256", "kernel": "gemm_sp_pair", "traffic_bytes": 7,
+         "family_src_hash": cur},
+        {"workload": "v", "plan": "pair256", "kernel": "gemm_sp_pair", "traffic_bytes": 9,
+         "family_src_hash": "0" * 16}]}))
+    assert bench.gemm_traffic("w", "pair256", str(p)) == 7
+    assert bench.gemm_traffic("v", "pair256", str(p)) is None
+
+
+def test_peaks_and_bytes():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    assert bench.sparse_peak(peaks, False, False) == 3200.0
+    assert bench.sparse_peak(peaks, False, True) == 2800.0
+    assert bench.sparse_peak(peaks, True, False) == 6400.0
+    # X + values + metadata + Y for bf16; int8 halves X and the values
+    assert bench.gemm_bytes(16, 64, 128, False) == 2 * 16 * 128 + 64 * 128 + 64 * 16 + 2 * 16 * 64
+    assert bench.gemm_bytes(16, 64, 128, True) == 16 * 128 + 64 * 64 + 64 * 16 + 2 * 16 * 64 + 256
+
+
+def test_oracle_sample_is_bounded_and_extrapolates():
+    # the CPU baseline on a slice of the largest configuration stays within
+    # its budget and reports the flops of a whole step
+    from structured_sparse_gemm_sp24_b200 import inputs as I
+    wl = I.Workload("cut", W=I.normal_bf16((16384, 1024), 1.0, 0),
+                    X=I.normal_bf16((16384, 1024), 1.0, 1))
+    import time
+    t0 = time.perf_counter()
+    flops, secs, sample, cores = bench.oracle_sample(wl, 0.3)
+    assert time.perf_counter() - t0 < 5.0
+    assert flops == 2.0 * 16384 * 16384 * 1024 and secs > 0 and cores >= 1
+    assert "extrapolated" in sample
+    # a small problem is done whole
+    small = I.Workload("tiny", W=I.normal_bf16((64, 128), 1.0, 0),
+                       X=I.normal_bf16((16, 128), 1.0, 1))
+    assert "whole step" in bench.oracle_sample(small, 5.0)[2]
 
 
 def _rank_main(rank, world, port, out):
