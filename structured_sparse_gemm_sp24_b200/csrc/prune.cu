@@ -247,6 +247,7 @@ constexpr int kStreamStage = kWTile + kMTile + kNTile + kSTile;   // multiple of
 constexpr int kStreamSmem = kStreamStages * kStreamStage + 4 * 2048 + 256 + 1024;
 constexpr int kXcTile = 128 * 256;   // fused Wanda norms: 128 tokens x 128 columns of Xc
 constexpr int kStreamSmemFused = kStreamSmem + kXcTile;
+constexpr int kProgExtra = 2 * 2048;   // progressive: staging of the first-stage mask
 
 struct StreamArgs {
   int64_t n, k;
@@ -256,6 +257,7 @@ struct StreamArgs {
   int mask_tma;                // the chunk's mask bytes come with the TMA stage
   const uint8_t* mask_direct;  // else read from here (NULL: no mask / mask_in)
   uint8_t* mask_out;           // NULL: not written
+  uint8_t* mask1_out;          // progressive: first-stage (3 of 4) mask, NULL: not written
   void* vals;
   uint8_t* meta;
   // Wanda with the column norms computed in the kernel (xc != NULL): each CTA
@@ -266,7 +268,11 @@ struct StreamArgs {
   double* norms_out;
 };
 
-template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
+//   kProg: progressive pruning in one pass ([Ampere-sparsity] Figure 4): the
+//          first-stage mask keeps 3 of 4, the second keeps 2 of 4 of the weights
+//          the first stage kept (dropped ones score 0); the second mask drives
+//          the values and metadata.  kPrune must be set and kMaskIn clear.
+template <bool kPrune, bool kWanda, int kVals, bool kMaskIn, bool kProg = false>
 __global__ void __launch_bounds__(kStreamThreads, 1)
 stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_mask,
               const __grid_constant__ CUtensorMap tm_norm, const __grid_constant__ CUtensorMap tm_sw,
@@ -278,7 +284,9 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
                                              ~uintptr_t(1023));
   uint8_t* meta_buf = smem + kStreamStages * kStreamStage;     // 2 x 2048
   uint8_t* mout_buf = meta_buf + 2 * 2048;                     // 2 x 2048
-  uint64_t* full = reinterpret_cast<uint64_t*>(mout_buf + 2 * 2048);
+  uint8_t* mout1_buf = mout_buf + 2 * 2048;                    // 2 x 2048 (kProg only)
+  uint64_t* full = reinterpret_cast<uint64_t*>(mout_buf + 2 * 2048 + (kProg ? kProgExtra : 0));
+  static_assert(!kProg || (kPrune && !kMaskIn), "progressive pruning computes its own masks");
 
   const int tid = threadIdx.x;
   const uint32_t bb = tid & 15u;              // vector within a chunk row
@@ -327,6 +335,7 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     const bool kv_ok = kv < kvec && ready;
     uint8_t* mb = meta_buf + (i & 1) * 2048;
     uint8_t* ob = mout_buf + (i & 1) * 2048;
+    uint8_t* ob1 = mout1_buf + (i & 1) * 2048;
     double nrm[8];
     if constexpr (kWanda) {
       if (fused_norms) {
@@ -404,7 +413,26 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
           }
         }
         uint32_t lo0, hi0, lo1, hi1;
-        if constexpr (kPrune && !kWanda && kVals != kValsNone) {
+        if constexpr (kProg) {
+          // stage 1 keeps 3 of 4; stage 2 keeps 2 of 4 of what stage 1 kept
+          uint32_t k3;
+          if constexpr (kWanda) {
+            k3 = mask_byte<true>(q, 0xFFu, nrm, 3);
+            keep = mask_byte<true>(q, k3, nrm, 2);
+          } else {
+            k3 = keep_nibble_mag<false>(q.x, q.y, 0xFu, 3) |
+                 (keep_nibble_mag<false>(q.z, q.w, 0xFu, 3) << 4);
+            keep = keep_nibble_mag<true>(q.x, q.y, k3 & 15u, 2) |
+                   (keep_nibble_mag<true>(q.z, q.w, k3 >> 4, 2) << 4);
+          }
+          if (a.mask1_out) ob1[m0 * 16 + bb + 512 * j] = static_cast<uint8_t>(k3);
+          if constexpr (kVals != kValsNone) {
+            uint32_t badv = 0;
+            const uint32_t c0 = nibble_code(keep & 15u, badv);
+            const uint32_t c1 = nibble_code(keep >> 4, badv);
+            lo0 = c0 & 3u; hi0 = c0 >> 2; lo1 = c1 & 3u; hi1 = c1 >> 2;
+          }
+        } else if constexpr (kPrune && !kWanda && kVals != kValsNone) {
           top2_positions_mag<kMaskIn>(q.x, q.y, mbyte & 15u, lo0, hi0);
           top2_positions_mag<kMaskIn>(q.z, q.w, mbyte >> 4, lo1, hi1);
           if (a.mask_out) keep = (1u << lo0) | (1u << hi0) | (((1u << lo1) | (1u << hi1)) << 4);
@@ -461,17 +489,21 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         __stcs(dst + tid, reinterpret_cast<const uint4*>(mb)[tid]);
       }
     }
-    if (a.mask_out && tid >= 256 && tid < 384) {
-      const int m = tid - 256;
+    // mask rows of the chunk: threads 256..383 the (second-stage) mask,
+    // threads 384..511 the first-stage mask of the progressive kernel
+    uint8_t* const mdst = tid < 384 ? a.mask_out : a.mask1_out;
+    const uint8_t* const msrc = tid < 384 ? ob : ob1;
+    if (mdst && tid >= 256 && (kProg || tid < 384)) {
+      const int m = (tid - 256) & 127;
       const int64_t row = static_cast<int64_t>(rt) * 128 + m;
       const int64_t v0 = static_cast<int64_t>(kb) * 16;
       int nb = static_cast<int>(kvec - v0 < 16 ? kvec - v0 : 16);
       if (row < a.n && nb > 0) {
-        uint8_t* dst = a.mask_out + row * kvec + v0;
+        uint8_t* dst = mdst + row * kvec + v0;
         if (nb == 16 && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
-          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(ob + m * 16);
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(msrc + m * 16);
         } else {
-          for (int e = 0; e < nb; ++e) dst[e] = ob[m * 16 + e];
+          for (int e = 0; e < nb; ++e) dst[e] = msrc[m * 16 + e];
         }
       }
     }
@@ -1150,15 +1182,16 @@ static sp24_status launch_colnorm(const void* xc, int64_t mc, int64_t k, double*
                        static_cast<const uint16_t*>(xc), mc, k, norms);
 }
 
-template <bool kPrune, bool kWanda, int kVals, bool kMaskIn>
+template <bool kPrune, bool kWanda, int kVals, bool kMaskIn, bool kProg = false>
 static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* mask_out,
                                  const double* norms, const float* s_w, int64_t n, int64_t k,
                                  int n_keep, void* vals, void* meta, cudaStream_t s,
-                                 const void* xc, int64_t mc) {
-  auto kern = stream_kernel<kPrune, kWanda, kVals, kMaskIn>;
+                                 const void* xc, int64_t mc, uint8_t* mask1_out = nullptr) {
+  auto kern = stream_kernel<kPrune, kWanda, kVals, kMaskIn, kProg>;
+  constexpr int kExtra = kProg ? kProgExtra : 0;
   static std::atomic<uint64_t> smem_set{0};   // one bit per device
   SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern),
-                         kWanda ? kStreamSmemFused : kStreamSmem, smem_set));
+                         (kWanda ? kStreamSmemFused : kStreamSmem) + kExtra, smem_set));
   cudaError_t e = cudaSuccess;
   const int64_t kblocks = (k + 127) / 128;
   const int64_t nchunks = ((n + 127) / 128) * kblocks;
@@ -1189,12 +1222,13 @@ static sp24_status launch_stream_t(const void* w, const uint8_t* mask, uint8_t* 
   a.mask_tma = mask_tma ? 1 : 0;
   a.mask_direct = mask_tma ? nullptr : mask;
   a.mask_out = mask_out;
+  a.mask1_out = mask1_out;
   a.vals = vals;
   a.meta = static_cast<uint8_t*>(meta);
   a.xc = static_cast<const uint16_t*>(xc);
   a.mc = mc;
   a.norms_out = const_cast<double*>(norms);
-  const int smem = (kWanda && xc != nullptr) ? kStreamSmemFused : kStreamSmem;
+  const int smem = ((kWanda && xc != nullptr) ? kStreamSmemFused : kStreamSmem) + kExtra;
   // as many persistent CTAs as fit (two per SM: one's barrier and TMA waits
   // overlap the other's work)
   int per_sm = 0;
@@ -1236,11 +1270,60 @@ static sp24_status launch_wanda_prune(const void* W, const uint8_t* mask_in, uin
                                               nullptr, nullptr, s);
 }
 
+// Progressive pruning in one pass (3 of 4, then 2 of 4 of the survivors),
+// optionally with the bf16 compression of the second mask.  Wanda norms as in
+// launch_wanda_prune.
+template <int kVals>
+static sp24_status launch_progressive(const void* W, int64_t N, int64_t K, const void* Xc,
+                                      int64_t Mc, bool wanda, uint8_t* mask1_out,
+                                      uint8_t* mask2_out, void* vals, void* meta, double* norms,
+                                      cudaStream_t s) {
+  if (!wanda)
+    return launch_stream_t<true, false, kVals, false, true>(W, nullptr, mask2_out, nullptr,
+                                                           nullptr, N, K, 2, vals, meta, s,
+                                                           nullptr, 0, mask1_out);
+  if (((N + 127) / 128) * Mc <= kFusedNormWork)
+    return launch_stream_t<true, true, kVals, false, true>(W, nullptr, mask2_out, norms, nullptr,
+                                                          N, K, 2, vals, meta, s, Xc, Mc,
+                                                          mask1_out);
+  SP24_TRY(launch_colnorm(Xc, Mc, K, norms, s));
+  return launch_stream_t<true, true, kVals, false, true>(W, nullptr, mask2_out, norms, nullptr, N,
+                                                        K, 2, vals, meta, s, nullptr, 0,
+                                                        mask1_out);
+}
+
 }  // namespace sp24
 
 using namespace sp24;
 
 extern "C" {
+
+sp24_status sp24_prune_progressive(const void* W, int64_t N, int64_t K, const void* Xc,
+                                   int64_t Mc, int mode, uint8_t* mask1_out, uint8_t* mask2_out,
+                                   void* vals, void* meta, void* workspace, void* stream) {
+  if (N < 0 || K < 0 || (mode != SP24_MAGNITUDE && mode != SP24_WANDA)) return SP24_ERR_ARG;
+  if (N == 0 || K == 0) return SP24_OK;
+  const bool compress = vals != nullptr || meta != nullptr;
+  if (!W || (compress && (!vals || !meta)) || (!compress && !mask1_out && !mask2_out))
+    return SP24_ERR_ARG;
+  if (mode == SP24_WANDA && (!Xc || Mc < 1 || !workspace)) return SP24_ERR_ARG;
+  if (K % (compress ? 16 : 8) != 0) return SP24_ERR_ALIGN;
+  if (!aligned16(W) || (mask1_out && !aligned16(mask1_out)) ||
+      (mask2_out && !aligned16(mask2_out)) || (vals && !aligned16(vals)) ||
+      (meta && !aligned16(meta)))
+    return SP24_ERR_ALIGN;
+  if (mode == SP24_WANDA && (!aligned16(Xc) || !aligned16(workspace))) return SP24_ERR_ALIGN;
+  if ((N + 127) / 128 > 65535) return SP24_ERR_ARG;
+  SP24_TRY(check_device());
+  cudaStream_t s = as_stream(stream);
+  double* norms = static_cast<double*>(workspace);
+  const bool wanda = mode == SP24_WANDA;
+  if (compress)
+    return launch_progressive<kValsBF16>(W, N, K, Xc, Mc, wanda, mask1_out, mask2_out, vals, meta,
+                                         norms, s);
+  return launch_progressive<kValsNone>(W, N, K, Xc, Mc, wanda, mask1_out, mask2_out, nullptr,
+                                       nullptr, norms, s);
+}
 
 sp24_status sp24_colnorm(const void* Xc, int64_t Mc, int64_t K, double* norms, void* stream) {
   if (!Xc || !norms || Mc < 1 || K < 1) return SP24_ERR_ARG;
