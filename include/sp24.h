@@ -257,6 +257,26 @@ sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
                                 uint8_t* mask_out, int dtype, const float* s_w,
                                 void* vals, void* meta, void* stream);
 
+/* Progressive pruning in one pass ([Ampere-sparsity] Figure 4: the 25 %
+ * stage keeps 3 of every 4 weights, the 50 % stage keeps 2 of 4 of the
+ * weights the first stage kept).  With no fine-tuning between the stages both
+ * masks come from the same weights, so one pass over W computes
+ *   mask1_out = the mask of sp24_prune(W, ..., n_keep = 3, mask_in = NULL)
+ *   mask2_out = the mask of sp24_prune(W, ..., n_keep = 2, mask_in = mask1)
+ * and, when vals and meta are given, the bf16 compression of W under mask2
+ * (the outputs of sp24_compress(W, mask2, SP24_BF16, ...)).
+ *   W: bf16 [N][K].  Xc, Mc, mode, workspace: as sp24_prune (for SP24_WANDA
+ *   the workspace holds the float64 column norms afterwards).
+ *   mask1_out, mask2_out: sp24_mask_bytes(N, K) bytes each, nullable.
+ *   vals, meta: both NULL (masks only) or both given (bf16 values [N][K/2],
+ *   sp24_meta_bytes(N, K) bytes of metadata).
+ * Rules: N >= 0, K % 8 == 0 (K % 16 == 0 with compression), at least one
+ * output; Mc >= 1 and a workspace for SP24_WANDA. */
+sp24_status sp24_prune_progressive(const void* W, int64_t N, int64_t K, const void* Xc,
+                                   int64_t Mc, int mode, uint8_t* mask1_out,
+                                   uint8_t* mask2_out, void* vals, void* meta,
+                                   void* workspace, void* stream);
+
 /* ----------------------------------------------------------- sparse GEMM */
 
 /* Y = X * W'^T with W' the 2:4 weight given by (vals, meta) ([Orin ch.7] 2.1
@@ -325,6 +345,36 @@ sp24_status sp24_gemm_plan(int64_t M, int64_t N, int64_t K, int dtype, sp24_gemm
  * Rules: B, H, W, C >= 0; elem_bytes in {1, 2}; C * elem_bytes % 16 == 0. */
 sp24_status sp24_im2col3x3(const void* X, int64_t B, int64_t H, int64_t W, int64_t C,
                            int elem_bytes, void* A, void* stream);
+
+/* 3x3 convolution as an implicit sparse GEMM ([Orin ch.7] 2.2 A.3: large
+ * 3x3 convolutions at large batch or high resolution are good 2:4
+ * candidates; 2.1: groups of 4 run along the input channels).  Stride 1, zero
+ * padding 1, NHWC:
+ *   Y[(b*H + h)*W + w][co] = sum_{kh, kw, c} X[b][h+kh-1][w+kw-1][c] * W'[co][kh][kw][c]
+ * with X zero outside the H x W image, i.e. sp24_gemm of the
+ * sp24_im2col3x3 operand, computed without forming that operand: the GEMM's
+ * token tiles are read straight from X (whole image rows per tile, the tap's
+ * shift in the load coordinates, the padding from the loads' zero fill).
+ *   X: [B][H][W][C] bf16 (dtype SP24_BF16) or int8 codes (SP24_INT8, from
+ *      sp24_quantize; a padded 0 is the code 0).
+ *   vals, meta: W[Cout][3][3][C] pruned and compressed as the [Cout][9*C]
+ *      matrix (sp24_prune / sp24_compress with K = 9*C; with C % 4 == 0
+ *      every group of 4 lies inside one tap).
+ *   s_x, s_w, out_kind, s_y, Y: as sp24_gemm with M = B*H*W and N = Cout;
+ *      Y is [B][H][W][Cout].
+ * Rules: C * element bytes % 128 == 0 (C % 64 == 0 for bf16, C % 128 == 0
+ * for int8), Cout % 8 == 0 (Cout % 16 == 0 for SP24_OUT_INT8), pointers
+ * 16-byte aligned.  Image rows must tile the GEMM's token tiles: there must be
+ * an r dividing H with (r * W) % 8 == 0 and r * W dividing 128 or 112 (e.g.
+ * W = 8, 16, 32, 56, 64, 112 or 128 with r = 1, or W = 28 with even H);
+ * otherwise the call returns SP24_ERR_UNSUPPORTED before any launch, and
+ * sp24_im2col3x3 followed by sp24_gemm computes the same convolution.  Up to
+ * 128 output channels run on single-SM tiles of 128 channels, more on CTA
+ * pairs of 256 channels. */
+sp24_status sp24_conv3x3(const void* X, int64_t B, int64_t H, int64_t W, int64_t C,
+                         const void* vals, const void* meta, int64_t Cout, int dtype,
+                         const float* s_x, const float* s_w, int out_kind, const float* s_y,
+                         void* Y, void* stream);
 
 /* ------------------------------------------------- allocation-free variant */
 

@@ -28,6 +28,13 @@ constexpr int kEpiWarps = 8;             // two per lane quadrant
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kEpiBox = 32;              // channels per warp store box
 
+// Threads of the persistent GEMM kernels: warp 0 producer, warp 1 MMA issuer,
+// warps 2..9 epilogue; the implicit convolution adds two warps (warp 10 a
+// second producer, warp 11 idle), which costs no registers: blocks are
+// allocated registers in whole groups of four warps.
+constexpr int kConvProducerWarp = 2 + kEpiWarps;
+__host__ __device__ constexpr int gemm_threads(bool conv) { return 64 + kEpiThreads + (conv ? 64 : 0); }
+
 template <int OUTK>
 struct EpiOut {
   static constexpr int kBytes = OUTK == SP24_OUT_INT32 ? 4 : (OUTK == SP24_OUT_INT8 ? 1 : 2);

@@ -60,8 +60,8 @@ __device__ __forceinline__ uint32_t make_idesc_pair(uint32_t id2) {
          (static_cast<uint32_t>(BN >> 3) << 17) | ((256u >> 4) << 24);
 }
 
-template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
-__global__ void __launch_bounds__(64 + kEpiThreads, 1)
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC, bool kConv = false>
+__global__ void __launch_bounds__(gemm_threads(kConv), 1)
 gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
              const __grid_constant__ CUtensorMap tmap_e, const __grid_constant__ CUtensorMap tmap_y,
              const __grid_constant__ CUtensorMap tmap_y16, const PersistArgs args) {
@@ -108,9 +108,12 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait_prior();   // set-up above overlapped the previous kernel's tail
 
-  if (warp == 0) {
+  if (warp == 0 || (kConv && warp == kConvProducerWarp)) {
     if (lane == 0) {
       // -------------------------------------------------------- producer
+      // (the implicit convolution runs two producer warps, each loading every
+      // other stage: its token loads take longer to issue)
+      const uint32_t pid = warp == 0 ? 0u : 1u;
       prefetch_tmap(&tmap_a);
       prefetch_tmap(&tmap_b);
       prefetch_tmap(&tmap_e);
@@ -119,8 +122,20 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         int prt, tt;
         tile_coords(tile, args, prt, tt);
         const int rt128 = prt * 2 + static_cast<int>(rank);   // this CTA's 128-row tile
+        ConvTileRows crow;
+        ConvTap ctap{0, 0};
+        if constexpr (kConv)
+          conv_tile_rows(static_cast<int64_t>(tt) * BN + static_cast<int>(rank) * C::kHalfN, args,
+                         crow);
         for (int kb = 0; kb < args.kblocks; ++kb, ++it) {
           const int s = it % STAGES;
+          if (kConv && (it & 1u) != pid) {   // the other producer's stage
+            if constexpr (kConv) {
+              ctap.advance(C::kLogicalK / 2, args.conv_c);
+              ctap.advance(C::kLogicalK / 2, args.conv_c);
+            }
+            continue;
+          }
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u)) { *abort_flag = 1; break; }
           uint8_t* st = smem + s * C::kStageStride;
@@ -129,9 +144,17 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
           tma_load_2d_pair(st, &tmap_a, fb, kb * (kDtype == SP24_BF16 ? 64 : 128), rt128 * 128);
           const int kx = kb * C::kLogicalK;
           const int ty = tt * BN + static_cast<int>(rank) * C::kHalfN;
-          tma_load_2d_pair(st + C::kABytes, &tmap_b, fb, kx, ty);
-          tma_load_2d_pair(st + C::kABytes + C::kBHalfBytes, &tmap_b, fb, kx + C::kLogicalK / 2,
-                           ty);
+          if constexpr (kConv) {
+            conv_load_tokens<C::kHalfN, C::kLogicalK>(
+                st + C::kABytes, ctap, crow, args,
+                [&](uint8_t* dst, int32_t c, int32_t w, int32_t h, int32_t b) {
+                  tma_load_4d_pair(dst, &tmap_b, fb, c, w, h, b);
+                });
+          } else {
+            tma_load_2d_pair(st + C::kABytes, &tmap_b, fb, kx, ty);
+            tma_load_2d_pair(st + C::kABytes + C::kBHalfBytes, &tmap_b, fb,
+                             kx + C::kLogicalK / 2, ty);
+          }
           // metadata map: 8 rows of 256 bytes per 2048-byte chunk
           tma_load_2d_pair(st + C::kABytes + 2 * C::kBHalfBytes, &tmap_e, fb, 0,
                            (rt128 * kchunks + kb * C::kMetaChunks) * 8);
@@ -186,7 +209,7 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
         if (aborted) break;
       }
     }
-  } else {
+  } else if (warp < 2 + kEpiWarps) {
     // --------------------------------------------------------- epilogue
     const int ew = warp - 2;                 // 0..7
     const int grp = ew >> 2;                 // which chunks of a tile (even / odd)
@@ -230,20 +253,29 @@ gemm_sp_pair(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__
 }
 
 // ------------------------------------------------------------ host launch
-template <int kDtype, int BN, int STAGES, int OUTK, int ACC>
+template <int kDtype, int BN, int STAGES, int OUTK, int ACC, bool kConv = false>
 sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x, int pairs,
-                        cudaStream_t s) {
+                        cudaStream_t s, const ConvGeom* cg = nullptr) {
   using C = PairCfg<kDtype, BN, STAGES, OUTK, ACC>;
-  auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC>;
+  auto kern = gemm_sp_pair<kDtype, BN, STAGES, OUTK, ACC, kConv>;
   static std::atomic<uint64_t> smem_set{0};   // one bit per device
   SP24_TRY(set_smem_once(reinterpret_cast<const void*>(kern), C::kSmemBytes, smem_set));
   const int el = kDtype == SP24_BF16 ? 2 : 1;
   const CUtensorMapDataType dt =
       kDtype == SP24_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  // B: each CTA loads BN/2 token rows
+  // B: each CTA loads BN/2 token rows (implicit convolution: boxes of whole
+  // image rows from the NHWC activations)
   CUtensorMap mb;
-  SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(g.k), static_cast<uint64_t>(g.m),
-                    static_cast<uint32_t>(128 / el), static_cast<uint32_t>(C::kHalfN)));
+  if constexpr (kConv) {
+    if (cg == nullptr) return SP24_ERR_ARG;
+    SP24_TRY(make_map_nhwc(&mb, x, dt, el, static_cast<uint64_t>(cg->c),
+                           static_cast<uint64_t>(cg->w), static_cast<uint64_t>(cg->h),
+                           static_cast<uint64_t>(cg->b), static_cast<uint32_t>(128 / el),
+                           static_cast<uint32_t>(cg->w), static_cast<uint32_t>(cg->rows)));
+  } else {
+    SP24_TRY(make_map(&mb, x, dt, el, static_cast<uint64_t>(g.k), static_cast<uint64_t>(g.m),
+                      static_cast<uint32_t>(128 / el), static_cast<uint32_t>(C::kHalfN)));
+  }
   // E: metadata chunks as rows of 256 bytes (8 rows per 2048-byte chunk)
   const int64_t kchunks = (g.k + 127) / 128;
   const int64_t rt128 = (g.n + 127) / 128;
@@ -278,16 +310,28 @@ sp24_status launch_pair(const CUtensorMap& ma, const GemmArgs& g, const void* x,
   a.kblocks = g.kblocks;
   a.row_tiles = static_cast<int>((g.n + 255) / 256);
   a.tok_tiles = static_cast<int>((g.m + BN - 1) / BN);
-  const int64_t row_tile_bytes = 256 * (g.k / 2) * el;
-  int64_t gr = (int64_t(24) << 20) / (row_tile_bytes > 0 ? row_tile_bytes : 1);
+  // raster band of 16 row-pair tiles: measured (ncu DRAM bytes per launch) on
+  // square 8192^3 and 16384^3 against bands of 3..32, it keeps both the band's
+  // weights and the token tiles of a wave in L2 best (16384^3: 10.2 GB read
+  // against 18.0 GB with 6)
+  int64_t gr = 16;
   gr = group_rows_override(gr);
   gr = gr < 1 ? 1 : (gr > a.row_tiles ? a.row_tiles : gr);
   a.group_rows = static_cast<int>(gr);
   a.y_box = y_box;
+  a.conv_h = a.conv_w = a.conv_c = a.conv_rows = a.conv_boxes = 0;
+  if constexpr (kConv) {
+    a.conv_h = static_cast<int>(cg->h);
+    a.conv_w = static_cast<int>(cg->w);
+    a.conv_c = static_cast<int>(cg->c);
+    a.conv_rows = cg->rows;
+    a.conv_boxes = cg->boxes;
+    if (cg->boxes * cg->rows * cg->w != C::kHalfN) return SP24_ERR_ARG;
+  }
   const int64_t ntiles = static_cast<int64_t>(a.row_tiles) * a.tok_tiles;
   if (ntiles > 0x7FFFFFFF) return SP24_ERR_UNSUPPORTED;
   if (pairs < 1 || pairs > ntiles) return SP24_ERR_ARG;   // the plan sizes the grid
-  return launch_kernel(kern, dim3(2 * pairs), dim3(64 + kEpiThreads), C::kSmemBytes, s, 2, ma,
+  return launch_kernel(kern, dim3(2 * pairs), dim3(gemm_threads(kConv)), C::kSmemBytes, s, 2, ma,
                        mb, me, my, my16, a);
 }
 

@@ -51,6 +51,31 @@ inline sp24_status make_map(CUtensorMap* map, const void* base, CUtensorMapDataT
   return cuda_fail("cuTensorMapEncodeTiled", buf);
 }
 
+// 4D map over an NHWC activation tensor [b][h][w][c] (dims innermost first:
+// c, w, h, b) with a {box_c, box_w, box_h, 1} box, 128-byte swizzle and zero
+// fill outside the tensor (the implicit convolution's padding).
+inline sp24_status make_map_nhwc(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
+                                 int elsize, uint64_t c, uint64_t w, uint64_t h, uint64_t b,
+                                 uint32_t box_c, uint32_t box_w, uint32_t box_h) {
+  if (!get_encoder()) return cuda_fail("cudaGetDriverEntryPoint", "cuTensorMapEncodeTiled");
+  const uint64_t es = static_cast<uint64_t>(elsize);
+  cuuint64_t dims[4] = {c, w, h, b};
+  cuuint64_t strides[3] = {c * es, w * c * es, h * w * c * es};
+  cuuint32_t box[4] = {box_c, box_w, box_h, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = tma_encoder()(map, dt, 4, const_cast<void*>(base), dims, strides, box, estr,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r == CUDA_SUCCESS) return SP24_OK;
+  char buf[112];
+  std::snprintf(buf, sizeof(buf), "CUresult %d (nhwc box %ux%ux%u, dims %llux%llux%llux%llu)",
+                static_cast<int>(r), box_c, box_w, box_h, static_cast<unsigned long long>(c),
+                static_cast<unsigned long long>(w), static_cast<unsigned long long>(h),
+                static_cast<unsigned long long>(b));
+  return cuda_fail("cuTensorMapEncodeTiled", buf);
+}
+
 // 1D map over `len` elements with a `box`-element box, zero fill past the end.
 inline sp24_status make_map_1d(CUtensorMap* map, const void* base, CUtensorMapDataType dt,
                                uint64_t len, uint32_t box) {

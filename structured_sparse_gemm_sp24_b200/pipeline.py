@@ -85,6 +85,22 @@ def prune_compress(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE,
     return (vals, meta, mask) if want_mask else (vals, meta)
 
 
+def prune_progressive(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE,
+                      Xc: Optional[torch.Tensor] = None, compress: bool = True):
+    """Progressive pruning in one pass: (mask1 keeping 3 of 4, mask2 keeping 2 of
+    4 of the survivors, vals, meta); vals and meta are None without
+    compression."""
+    N, K = W.shape
+    mask1 = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    mask2 = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    vals = meta = None
+    if compress:
+        vals, meta = alloc_compressed(N, K, _b.SP24_BF16, W.device)
+    ws = _u8(max(_b.sp24_prune_workspace_bytes(K, mode), 16), W.device)
+    _b.sp24_prune_progressive(W, Xc, mode, mask1, mask2, vals, meta, ws)
+    return mask1, mask2, vals, meta
+
+
 def gemm(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, N: int,
          dtype: int = _b.SP24_BF16, s_x: Optional[torch.Tensor] = None,
          s_w: Optional[torch.Tensor] = None, out_kind: int = _b.SP24_OUT_BF16,
@@ -133,9 +149,25 @@ def im2col3x3(X: torch.Tensor) -> torch.Tensor:
 
 
 def conv3x3(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, Cout: int,
-            **gemm_kwargs) -> torch.Tensor:
+            dtype: int = _b.SP24_BF16, s_x: Optional[torch.Tensor] = None,
+            s_w: Optional[torch.Tensor] = None, out_kind: int = _b.SP24_OUT_BF16,
+            s_y: Optional[torch.Tensor] = None, path: str = "auto") -> torch.Tensor:
     """3x3 convolution (stride 1, padding 1) of NHWC X with 2:4 weights
-    compressed from W[Cout][3][3][C] viewed as [Cout][9*C].  Returns NHWC Y."""
+    compressed from W[Cout][3][3][C] viewed as [Cout][9*C].  Returns NHWC Y.
+
+    path "implicit": sp24_conv3x3 (token tiles read straight from X);
+    "explicit": sp24_im2col3x3 then sp24_gemm; "auto": implicit where its
+    tiling rules allow, else explicit."""
     Bn, H, W, _ = X.shape
-    y = gemm(im2col3x3(X), vals, meta, Cout, **gemm_kwargs)
+    odt = {_b.SP24_OUT_BF16: torch.bfloat16, _b.SP24_OUT_INT32: torch.int32,
+           _b.SP24_OUT_INT8: torch.int8}[out_kind]
+    if path in ("auto", "implicit"):
+        y = torch.empty((Bn, H, W, Cout), dtype=odt, device=X.device)
+        try:
+            _b.sp24_conv3x3(X, vals, meta, Cout, dtype, s_x, s_w, out_kind, s_y, y)
+            return y
+        except _b.Sp24Error as e:
+            if path == "implicit" or e.status not in (_b.SP24_ERR_UNSUPPORTED, _b.SP24_ERR_ALIGN):
+                raise
+    y = gemm(im2col3x3(X), vals, meta, Cout, dtype, s_x, s_w, out_kind, s_y)
     return y.view(Bn, H, W, Cout)

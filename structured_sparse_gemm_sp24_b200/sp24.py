@@ -58,6 +58,10 @@ SIGNATURES = {
     "sp24_compress": (_c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p, _c_p]),
     "sp24_prune_compress": (_c_int, [_c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p, _c_int,
                                      _c_p, _c_p, _c_p, _c_p]),
+    "sp24_prune_progressive": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_int, _c_p, _c_p,
+                                        _c_p, _c_p, _c_p, _c_p]),
+    "sp24_conv3x3": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_int,
+                              _c_p, _c_p, _c_int, _c_p, _c_p, _c_p]),
     "sp24_gemm": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_int, _c_p, _c_p, _c_int,
                            _c_p, _c_p, _c_p]),
     "sp24_device_status": (_c_int, [_c_p]),
@@ -237,6 +241,26 @@ def sp24_prune_compress(W: torch.Tensor, mode: int, norms: Optional[torch.Tensor
     _check(lib().sp24_prune_compress(_ptr(W), N, K, mode, _ptr(norms), _ptr(mask_in),
                                      _ptr(mask_out), dtype, _ptr(s_w), _ptr(vals), _ptr(meta),
                                      _stream(stream)), "sp24_prune_compress")
+
+
+def sp24_prune_progressive(W: torch.Tensor, Xc: Optional[torch.Tensor], mode: int,
+                           mask1_out: Optional[torch.Tensor], mask2_out: Optional[torch.Tensor],
+                           vals: Optional[torch.Tensor], meta: Optional[torch.Tensor],
+                           workspace: Optional[torch.Tensor], stream=None) -> None:
+    N, K = W.shape
+    Mc = Xc.shape[0] if Xc is not None else 0
+    _check(lib().sp24_prune_progressive(_ptr(W), N, K, _ptr(Xc), Mc, mode, _ptr(mask1_out),
+                                        _ptr(mask2_out), _ptr(vals), _ptr(meta), _ptr(workspace),
+                                        _stream(stream)), "sp24_prune_progressive")
+
+
+def sp24_conv3x3(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, Cout: int, dtype: int,
+                 s_x: Optional[torch.Tensor], s_w: Optional[torch.Tensor], out_kind: int,
+                 s_y: Optional[torch.Tensor], Y: torch.Tensor, stream=None) -> None:
+    Bn, H, W, C = X.shape
+    _check(lib().sp24_conv3x3(_ptr(X), Bn, H, W, C, _ptr(vals), _ptr(meta), Cout, dtype,
+                              _ptr(s_x), _ptr(s_w), out_kind, _ptr(s_y), _ptr(Y),
+                              _stream(stream)), "sp24_conv3x3")
 
 
 def sp24_gemm(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, N: int, dtype: int,

@@ -188,3 +188,49 @@ def test_im2col_host_validation(lib):
     assert f(FAKE, 1, 4, 4, 12, 2, FAKE, None) == B.SP24_ERR_ALIGN  # 24-byte pixels
     assert f(FAKE, 1, 4, 4, 8, 1, FAKE, None) == B.SP24_ERR_ALIGN   # 8-byte pixels
     assert f(FAKE + 8, 1, 4, 4, 8, 2, FAKE, None) == B.SP24_ERR_ALIGN
+
+
+def test_prune_progressive_host_validation(lib):
+    f = lib.sp24_prune_progressive
+    M, W_ = B.SP24_MAGNITUDE, B.SP24_WANDA
+    # no output at all
+    assert f(FAKE, 8, 16, None, 0, M, None, None, None, None, None, None) == B.SP24_ERR_ARG
+    # values without metadata (or the reverse)
+    assert f(FAKE, 8, 16, None, 0, M, FAKE, None, FAKE, None, None, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 8, 16, None, 0, M, FAKE, None, None, FAKE, None, None) == B.SP24_ERR_ARG
+    # unknown mode; wanda without calibration rows or workspace
+    assert f(FAKE, 8, 16, None, 0, 9, FAKE, None, None, None, None, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 8, 16, None, 4, W_, FAKE, None, None, None, FAKE, None) == B.SP24_ERR_ARG
+    assert f(FAKE, 8, 16, FAKE, 4, W_, FAKE, None, None, None, None, None) == B.SP24_ERR_ARG
+    # K: multiple of 8 for masks, of 16 with compression
+    assert f(FAKE, 8, 12, None, 0, M, FAKE, None, None, None, None, None) == B.SP24_ERR_ALIGN
+    assert f(FAKE, 8, 24, None, 0, M, FAKE, FAKE, FAKE, FAKE, None, None) == B.SP24_ERR_ALIGN
+    # misaligned pointers
+    assert f(FAKE + 2, 8, 16, None, 0, M, FAKE, None, None, None, None, None) == B.SP24_ERR_ALIGN
+    assert f(FAKE, 8, 16, None, 0, M, FAKE + 4, None, None, None, None, None) == B.SP24_ERR_ALIGN
+    # empty problem
+    assert f(None, 0, 16, None, 0, M, None, None, None, None, None, None) == B.SP24_OK
+
+
+def test_conv3x3_host_validation(lib):
+    f = lib.sp24_conv3x3
+    BF, I8 = B.SP24_BF16, B.SP24_INT8
+    OB, O32, O8 = B.SP24_OUT_BF16, B.SP24_OUT_INT32, B.SP24_OUT_INT8
+    ok = (FAKE, 2, 8, 16, 64, FAKE, FAKE, 64, BF, None, None, OB, None, FAKE, None)
+    def call(**kw):
+        names = ["X", "B", "H", "W", "C", "vals", "meta", "Cout", "dtype", "s_x", "s_w",
+                 "out", "s_y", "Y", "stream"]
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return f(*[a[n] for n in names])
+    assert call(dtype=5) == B.SP24_ERR_ARG
+    assert call(out=O32) == B.SP24_ERR_ARG               # bf16 has only a bf16 output
+    assert call(dtype=I8, C=128, out=OB) == B.SP24_ERR_ARG   # dequant needs the scales
+    assert call(dtype=I8, C=128, out=O8, s_x=FAKE, s_w=FAKE) == B.SP24_ERR_ARG   # and s_y
+    assert call(C=32) == B.SP24_ERR_ALIGN                # 64-byte channel rows
+    assert call(dtype=I8, C=64, out=O32) == B.SP24_ERR_ALIGN
+    assert call(Cout=60) == B.SP24_ERR_ALIGN
+    assert call(X=FAKE + 8) == B.SP24_ERR_ALIGN
+    assert call(meta=None) == B.SP24_ERR_ARG
+    assert call(B=-1) == B.SP24_ERR_ARG
+    assert call(B=0) == B.SP24_OK and call(Cout=0) == B.SP24_OK

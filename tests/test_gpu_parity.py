@@ -135,6 +135,41 @@ def test_progressive_bert():
     assert np.array_equal(keep_of(m2, w.K), r2)
 
 
+# (N, K, Mc): fused-norm path (BERT fc1), ragged K tail with a partial row
+# tile, and the separate column-norm kernel (82 row tiles x 128 rows > 8192)
+PROGRESSIVE_SHAPES = [(3072, 768, 128), (200, 136, 37), (10400, 256, 128)]
+
+
+@pytest.mark.parametrize("mode", [B.SP24_WANDA, B.SP24_MAGNITUDE])
+@pytest.mark.parametrize("nkm", PROGRESSIVE_SHAPES)
+def test_prune_progressive_one_pass(mode, nkm):
+    # one pass: mask1 (3 of 4), mask2 (2 of 4 on W * mask1), bf16 values and
+    # metadata of mask2, bit for bit against the oracle's two-stage definition
+    n, k, mc = nkm
+    W = I.normal_bf16((n, k), 0.02, seed=61)
+    Xc = I.normal_bf16((mc, k), 1.0, seed=62)
+    xc = Xc.cuda() if mode == B.SP24_WANDA else None
+    omode = O.WANDA if mode == B.SP24_WANDA else O.MAGNITUDE
+    r1, r2 = O.progressive(f64(W), omode, f64(Xc) if mode == B.SP24_WANDA else None)
+    compress = k % 16 == 0
+    m1, m2, vals, meta = P.prune_progressive(W.cuda(), mode, xc, compress=compress)
+    ok_status()
+    assert np.array_equal(keep_of(m1, k), r1)
+    assert np.array_equal(keep_of(m2, k), r2)
+    if compress:
+        rv, rm = O.compress(f64(W), r2)
+        assert np.array_equal(f64(vals), rv)
+        assert np.array_equal(canon_meta(meta, n, k, L.BF16), rm)
+    # masks only, one output at a time
+    m1b = torch.empty_like(m1)
+    ws = torch.empty(max(B.sp24_prune_workspace_bytes(k, mode), 16), dtype=torch.uint8,
+                     device="cuda")
+    B.sp24_prune_progressive(W.cuda(), xc, mode, m1b, None, None, None, ws)
+    assert torch.equal(m1b, m1)
+    if mode == B.SP24_WANDA:   # the workspace holds the column norms afterwards
+        assert np.array_equal(ws[: 8 * k].view(torch.float64).cpu().numpy(), O.column_norms(f64(Xc)))
+
+
 def test_prune_llm_full():
     w = I.llm_proj(11008, 4096, 16)
     mask = P.prune(w.W.cuda(), B.SP24_MAGNITUDE, 2)
