@@ -2,9 +2,10 @@
 """Benchmark of the 2:4 sparse path on B200 (one JSON line on rank 0).
 
 A step is one pass of the whole path over one batch of synthetic input:
-  bf16 workloads:  [Wanda: column norms] -> prune (3:4 stage for the
-                   progressive workload) -> fused prune+compress 2:4 ->
-                   sparse GEMM Y = X * W'^T
+  bf16 workloads:  [Wanda: column norms] -> fused prune+compress 2:4 ->
+                   sparse GEMM Y = X * W'^T; the progressive (BERT fc1)
+                   workload forms the 3:4 mask, the 2:4 mask on its
+                   survivors and the compressed operand in one pass
   int8 workload:   prune 2:4 -> per-channel scale -> compress to int8 ->
                    per-tensor activation scale -> quantise X -> int8 sparse
                    GEMM with bf16 dequantisation.
@@ -15,7 +16,8 @@ whole step time; the roofline of the dominant kernel (the GEMM) is reported
 beside it, and a `configs` block gives the GEMM and prune/compress figures of
 every other configured workload (BERT fc1, LLM projections at M = 16, 128 and
 2048, INT8, square 4096 / 8192, the 1x1 convolution).  Inputs are resident in
-HBM; L2 is flushed between timed steps by writing a 512 MB buffer.
+HBM; L2 is flushed between timed steps by writing a 512 MB buffer and reading
+it back (so the flush's own write-back is not charged to the next kernel).
 
 Multi-GPU: one process per GPU (torchrun), each rank runs an independent
 replica of the workload (weak scaling); time = max over ranks.
@@ -55,6 +57,16 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_SUSTAINED = 1400.0
 L2_FLUSH_BYTES = 512 << 20
+
+
+def flush_l2(buf: torch.Tensor) -> None:
+    """Evicts the workload's data from L2 (126 MB) before a timed step: writes
+    the 512 MB buffer, then reads it back, so that the write-back of the
+    flush's own dirty lines happens here and not inside the next timed
+    kernel (a write-only flush leaves ~126 MB of dirty lines whose eviction
+    the next HBM-bound kernel would pay for)."""
+    buf.zero_()
+    buf.view(torch.int32).sum()
 TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
 
 
@@ -174,6 +186,8 @@ class Runner:
             # the library forms the column norms inside the prune kernel when
             # row tiles x calibration rows is small, else launches colnorm first
             fused = ((self.N + 127) // 128) * self.wl.Xc.shape[0] <= 8192
+            if self.wl.progressive:
+                return (1 if fused else 2) + 1       # [colnorm +] progressive prune, gemm
             return (1 if fused else 2) + 1 + 1   # [colnorm +] prune, prune_compress, gemm
         return 1 + 1                         # prune_compress, gemm
 
@@ -193,13 +207,21 @@ class Runner:
             rec(2)
             B.sp24_gemm(self.Xq, self.vals, self.meta, self.N, B.SP24_INT8, self.s_x, self.s_w,
                         B.SP24_OUT_BF16, None, self.Y)
+        elif self.wanda and wl.progressive:
+            # one pass: norms, the 3:4 mask, the 2:4 mask on the survivors and
+            # the compressed operand
+            rec(1)
+            B.sp24_prune_progressive(self.W, self.Xc, B.SP24_WANDA, self.mask1, self.mask2,
+                                     self.vals, self.meta, self.ws)
+            rec(2)
+            B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
+                        B.SP24_OUT_BF16, None, self.Y)
         elif self.wanda:
             # prune also leaves the float64 column norms in its workspace
-            n_keep = 3 if wl.progressive else 2
+            n_keep = 2
             B.sp24_prune(self.W, self.Xc, B.SP24_WANDA, n_keep, None, self.mask1, self.ws)
             rec(1)
-            B.sp24_prune_compress(self.W, B.SP24_WANDA, self.ws,
-                                  self.mask1 if wl.progressive else None, None, B.SP24_BF16,
+            B.sp24_prune_compress(self.W, B.SP24_WANDA, self.ws, None, None, B.SP24_BF16,
                                   None, self.vals, self.meta)
             rec(2)
             B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
@@ -227,8 +249,11 @@ class Runner:
             # compress int8: read W + mask, write values + metadata; the
             # activation scale passes and quantisation share the stage
             return 2 * N * K + N * K / 8 + N * K / 2 + N * K / 8
-        extra = N * K / 8 if self.wl.progressive else 0   # mask_in
-        return 2 * N * K + extra + N * K + N * K / 8
+        if self.wl.progressive:
+            # one pass: read W (and Xc), write both masks, values and metadata
+            mc = self.wl.Xc.shape[0] if self.wl.Xc is not None else 0
+            return 2 * mc * K + 2 * N * K + 2 * N * K / 8 + N * K + N * K / 8
+        return 2 * N * K + N * K + N * K / 8
 
     def prune_bytes(self) -> float:
         N, K = self.N, self.K
@@ -258,8 +283,8 @@ def workload_config(wl: I.Workload, world: int) -> dict:
     """The `config` object of a JSON line (same for both arms)."""
     return {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K, "mode": wl.mode,
             "progressive": wl.progressive, "int8": wl.int8,
-            "l2": "flushed between steps (512 MB write); W, X, Y also exceed L2"
-            if wl.M * wl.K * 2 > (126 << 20) else "flushed between steps (512 MB write)",
+            "l2": ("flushed between steps (512 MB written then read back)"
+                   + ("; W, X, Y also exceed L2" if wl.M * wl.K * 2 > (126 << 20) else "")),
             "parallelism": f"replicas{world}"}
 
 
@@ -325,7 +350,7 @@ def time_steps(runner, steps, flush, use_graph=True, stage_steps=None):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(steps)]
         for i in range(steps):
-            flush.zero_()
+            flush_l2(flush)
             ev[i][0].record()
             graph.replay()
             ev[i][1].record()
@@ -343,7 +368,7 @@ def time_steps(runner, steps, flush, use_graph=True, stage_steps=None):
             graphs.append(g)
         torch.cuda.synchronize()
     for i in range(stage_steps):
-        flush.zero_()
+        flush_l2(flush)
         if use_graph:
             graphs[i].replay()
         else:
@@ -453,7 +478,7 @@ def measure_config(name, device, flush, peaks, steps):
     wl = I.by_name(name)
     runner = Runner(wl, device)
     for _ in range(3):
-        flush.zero_()
+        flush_l2(flush)
         runner.step()
     torch.cuda.synchronize()
     tot, prune, comp, gemm = time_steps(runner, steps, flush)
@@ -502,7 +527,10 @@ def oracle_sample(wl: I.Workload, budget_s: float):
     mode = O.WANDA if wl.mode == "wanda" else O.MAGNITUDE
     done_w, t_prune, last = 0, 0.0, 0   # rows pruned in all slices, time, largest slice
     vals = meta = s_w = None
-    while last < n and (last == 0 or t_prune < 0.4 * budget_s):
+    t_last = 0.0
+    # the next slice (twice the rows) takes about twice as long: start it only
+    # if it still fits 40 % of the budget
+    while last < n and (last == 0 or t_prune + 2.0 * t_last < 0.4 * budget_s):
         r = min(2 * last if last else 64, n)
         w = wl.W[:r].to(torch.float64).numpy()
         t0 = time.perf_counter()
@@ -513,23 +541,33 @@ def oracle_sample(wl: I.Workload, budget_s: float):
         else:
             keep = O.progressive(w, mode, xc)[1] if wl.progressive else O.prune(w, mode, 2, xc=xc)
             vals, meta = O.compress(w, keep)
-        t_prune += time.perf_counter() - t0
+        t_last = time.perf_counter() - t0
+        t_prune += t_last
         done_w += r
         last = r
-    x_rows, t_gemm, r = 0, 0.0, 8
-    while x_rows < m and (x_rows == 0 or t_prune + t_gemm < budget_s):
-        r = min(r, m - x_rows)
-        t1 = time.perf_counter()
+    def gemm_rows(r):
         if wl.int8:
-            x = wl.X[x_rows:x_rows + r].numpy()
+            x = wl.X[:r].numpy()
             s_x = O.tensor_scale(x)   # per-sample scale: same arithmetic, bounded cost
             acc = O.gemm_int8_acc(O.quantize(x, s_x), vals, meta, k)
             O.dequant_bf16(acc, s_x, s_w)
         else:
-            O.gemm(wl.X[x_rows:x_rows + r].to(torch.float64).numpy(), vals, meta, k)
-        t_gemm += time.perf_counter() - t1
-        x_rows += r
-        r *= 2
+            O.gemm(wl.X[:r].to(torch.float64).numpy(), vals, meta, k)
+
+    # a probe of 16 rows sizes one call that fills the rest of the budget (the
+    # oracle rebuilds the dense weight on every call, so one large call is
+    # timed rather than many small ones)
+    r = min(16, m)
+    t1 = time.perf_counter()
+    gemm_rows(r)
+    t_probe = time.perf_counter() - t1
+    x_rows, t_gemm = r, t_probe
+    left = budget_s - t_prune - t_probe
+    if x_rows < m and left > 0:
+        r = int(min(m, max(16, left / max(t_probe, 1e-9) * 16)))
+        t1 = time.perf_counter()
+        gemm_rows(r)
+        x_rows, t_gemm = r, time.perf_counter() - t1
     step_s = t_prune / done_w * n + t_gemm / (x_rows * last) * m * n
     cores = None
     for info in threadpoolctl.threadpool_info():
@@ -657,7 +695,7 @@ def main(argv=None):
     runner = Runner(wl, device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2(flush)
         runner.step()
     torch.cuda.synchronize()
     if B.sp24_device_status() != B.SP24_OK:
