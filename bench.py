@@ -198,6 +198,9 @@ class Runner:
         wl = self.wl
         rec(0)
         if wl.int8:
+            # (a second stream for the activation side was measured slower:
+            # its many small CTAs keep the weight-side persistent kernels off
+            # the SMs)
             B.sp24_prune(self.W, None, B.SP24_MAGNITUDE, 2, None, self.mask2, None)
             B.sp24_wscale(self.W, self.mask2, 0.9999, self.s_w)
             rec(1)
@@ -508,6 +511,67 @@ def measure_config(name, device, flush, peaks, steps):
     return out
 
 
+def time_graph(fn, flush, reps=10):
+    """Median CUDA-event time (ms) of one replay of a graph of `fn`, L2
+    flushed before each replay."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    ts = []
+    for _ in range(reps):
+        flush_l2(flush)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    del g
+    return statistics.median(ts)
+
+
+def measure_extras(device, flush, peaks):
+    """The rows after the path proper: the 3x3 convolution as an implicit GEMM
+    against the explicit gather + GEMM (ResNet stage-2 shape, batch 32), and
+    the Sparse-QAT forward fake-quantisation of the INT8 workload's weight."""
+    from structured_sparse_gemm_sp24_b200 import pipeline as P
+    out = {}
+    b, h, w, c, cout = 32, 28, 28, 128, 128
+    w4 = I.normal_bf16((cout, 3, 3, c), 0.05, 51).to(device)
+    x = I.normal_bf16((b, h, w, c), 1.0, 52).to(device)
+    vals, meta = P.prune_compress(w4.view(cout, 9 * c), B.SP24_MAGNITUDE)
+    a = torch.empty((b * h * w, 9 * c), dtype=torch.bfloat16, device=device)
+    y = torch.empty((b * h * w, cout), dtype=torch.bfloat16, device=device)
+    yi = torch.empty((b, h, w, cout), dtype=torch.bfloat16, device=device)
+    t_imp = time_graph(lambda: B.sp24_conv3x3(x, vals, meta, cout, B.SP24_BF16, None, None,
+                                              B.SP24_OUT_BF16, None, yi), flush)
+    t_exp = time_graph(lambda: (B.sp24_im2col3x3(x, a),
+                                B.sp24_gemm(a, vals, meta, cout, B.SP24_BF16, None, None,
+                                            B.SP24_OUT_BF16, None, y)), flush)
+    m, k = b * h * w, 9 * c
+    flops = 2.0 * m * cout * k
+    out["conv3x3"] = {"shape": f"NHWC {b}x{h}x{w}x{c} -> {cout}, 3x3, stride 1, pad 1",
+                      "implicit_us": 1e3 * t_imp, "explicit_gather_gemm_us": 1e3 * t_exp,
+                      "implicit_tflops_dense_equiv": flops / (t_imp * 1e-3) / 1e12,
+                      "speedup_vs_explicit": t_exp / t_imp}
+    wl = I.int8_long_tail()
+    W = wl.W.to(device)
+    mask = P.prune(W, B.SP24_MAGNITUDE, 2)
+    s_w = P.wscale(W, mask)
+    wfq = torch.empty_like(W)
+    t_fq = time_graph(lambda: B.sp24_fake_quant(W, mask, s_w, wfq), flush)
+    n, kk = W.shape
+    fq_bytes = 2 * n * kk + n * kk / 8 + 4 * n + 2 * n * kk
+    out["fake_quant"] = {"shape": f"W {n}x{kk}", "us": 1e3 * t_fq,
+                         "gbs": fq_bytes / (t_fq * 1e-3) / 1e9,
+                         "frac_hbm": fq_bytes / (t_fq * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+    if B.sp24_device_status() != B.SP24_OK:
+        raise SystemExit("device status not OK after the extra rows")
+    return out
+
+
 # ---------------------------------------------------------------- CPU oracle
 def oracle_sample(wl: I.Workload, budget_s: float):
     """Times the CPU oracle (as it stands) on a bounded sample of the workload
@@ -781,6 +845,7 @@ def main(argv=None):
     if world == 1 and not args.no_configs:
         line["configs"] = [measure_config(n, device, flush, peaks, args.config_steps)
                            for n in CONFIG_WORKLOADS if n != wl.name]
+        line["extras"] = measure_extras(device, flush, peaks)
     if world == 1 and not args.no_cpu_baseline:
         flops, secs, sample, cores = oracle_sample(wl, args.cpu_budget)
         line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores,

@@ -563,6 +563,7 @@ __global__ void __launch_bounds__(256) wscale_kernel(const uint16_t* __restrict_
   uint32_t* h = hist[wid];
 
   uint32_t cnt = 0, kmax = 0;
+#pragma unroll 4
   for (int64_t v = lane; v < kvec; v += 32) {
     const uint4 q = __ldg(reinterpret_cast<const uint4*>(wr) + v);
     const uint32_t keep = mr[v];
@@ -660,8 +661,19 @@ struct ActScaleWs {
   uint32_t ncand;        // keys in [lo, hi] (counts past the capacity)
   uint32_t done;         // 1 once s_x holds the answer
   uint32_t blocks_done;  // radix pass: CTAs finished (the last one selects)
+  uint32_t fine[4096];   // bracket pass: candidates per fine bin (see act_fine_bin)
   uint32_t cand[kActCandCap];
 };
+
+// Fine bin of a candidate key >= lo: 2048 bins per binary exponent over the
+// two exponents starting at lo's (the top 11 mantissa bits), keys beyond in
+// the last bin.  base = lo with its mantissa cleared.  Every key of a bin
+// b < 4095 agrees with base + (b << 12) on bits 12 and up.
+constexpr uint32_t kActFineBins = 4096;
+__device__ __forceinline__ uint32_t act_fine_bin(uint32_t key, uint32_t base) {
+  const uint32_t b = (key - base) >> 12;
+  return b < kActFineBins - 1 ? b : kActFineBins - 1;
+}
 
 // Inclusive prefix sum of v over a block of 1024 threads (scratch: 32 words).
 __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* scratch) {
@@ -812,6 +824,7 @@ __global__ void __launch_bounds__(1024) act_sample_select(int64_t count, uint32_
   if (excl < k_lo && k_lo <= incl) bins[0] = b0 + (k_lo > excl + h0 ? 1u : 0u);
   if (excl < k_hi && k_hi <= incl) bins[1] = b0 + (k_hi > excl + h0 ? 1u : 0u);
   __syncthreads();
+  for (int i = threadIdx.x; i < static_cast<int>(kActFineBins); i += blockDim.x) ws->fine[i] = 0;
   if (threadIdx.x == 0) {
     ws->lo = has_lo ? bins[0] << 20 : 0u;
     ws->hi = has_hi ? (bins[1] << 20) | 0xFFFFFu : 0xFFFFFFFFu;
@@ -891,6 +904,12 @@ __global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x,
   if (n <= kActLocalCap)
     for (uint32_t i = threadIdx.x; i < n; i += blockDim.x)
       if (base + i < kActCandCap) ws->cand[base + i] = buf[i];
+  // each candidate also counts in its fine bin (for the final selection)
+  if (n <= kActLocalCap) {
+    const uint32_t fbase = lo & 0x7F800000u;
+    for (uint32_t i = threadIdx.x; i < n; i += blockDim.x)
+      atomicAdd(&ws->fine[act_fine_bin(buf[i], fbase)], 1u);
+  }
 }
 
 // Candidates staged in dynamic shared memory when they fit (kActSelSmemKeys),
@@ -906,6 +925,66 @@ __global__ void __launch_bounds__(1024) act_bracket_select(ActScaleWs* ws, float
   const uint32_t below = ws->below, n = ws->ncand, rank = ws->rank;
   if (!(below < rank && rank - below <= n && n <= kActCandCap)) return;   // radix decides
   const uint32_t* cand = ws->cand;
+  // fine bin holding the (rank - below)-th candidate, from the bracket pass's
+  // histogram: 4 bins per thread, one block scan
+  {
+    const uint32_t k = rank - below;
+    uint32_t h[4], local = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      h[j] = __ldcg(ws->fine + 4 * threadIdx.x + j);
+      local += h[j];
+    }
+    const uint32_t incl = block_incl_scan(local, scratch);
+    uint32_t acc = incl - local;
+    if (acc < k && k <= incl) {
+      uint32_t b = 4 * threadIdx.x;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        if (acc + h[j] >= k) break;
+        acc += h[j];
+        ++b;
+      }
+      scratch[32] = b;
+      scratch[33] = acc;
+      scratch[31] = h[b - 4 * threadIdx.x];
+    }
+    __syncthreads();
+    const uint32_t bin = scratch[32], before = scratch[33], cnt = scratch[31];
+    __syncthreads();
+    // every key of a bin below the last agrees on bits 12 and up: select
+    // among that bin's candidates only
+    if (bin < kActFineBins - 1 && cnt <= kActSelSmemKeys) {
+      const uint32_t fbase = ws->lo & 0x7F800000u;
+      __shared__ uint32_t nsel;
+      if (threadIdx.x == 0) nsel = 0;
+      __syncthreads();
+      // eight loads in flight per thread, then the (rare) appends
+      constexpr int kU = 8;
+      for (uint32_t i0 = threadIdx.x; i0 < n; i0 += kU * blockDim.x) {
+        uint32_t v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const uint32_t i = i0 + u * blockDim.x;
+          v[u] = i < n ? __ldcg(cand + i) : 0xFFFFFFFFu;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          if (v[u] != 0xFFFFFFFFu && act_fine_bin(v[u], fbase) == bin)
+            ck[atomicAdd(&nsel, 1u)] = v[u];
+      }
+      __syncthreads();
+      const uint32_t fixed = fbase + (bin << 12);
+      const uint32_t key = block_select([&](uint32_t j) { return ck[j]; }, cnt, k - before, hist,
+                                        scratch, 12, fixed);
+      if (threadIdx.x == 0) {
+        const float t = __uint_as_float(key);
+        *s_x = (t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
+        ws->done = 1;
+      }
+      return;
+    }
+  }
   // every candidate lies in [lo, max]: only the bits below the highest bit in
   // which lo and the largest candidate differ can vary
   __shared__ uint32_t wmax[32];
