@@ -138,7 +138,7 @@ const char* sp24_strerror(int status) {
   }
 }
 
-int sp24_version(void) { return 200; }
+int sp24_version(void) { return 300; }
 
 const char* sp24_last_cuda_error(void) { return g_last_err; }
 

@@ -704,6 +704,10 @@ def test_gemm_plan_families(monkeypatch):
     assert big["ctas"] % 2 == 0 and 2 <= big["ctas"] <= sms
     conv = B.sp24_gemm_plan(200704, 64, 256, B.SP24_BF16)
     assert conv["kernel"] == "single" and conv["ctas"] == sms
+    # less than one wave of 128 x 128 tiles (86 for N = 11008): split-K
+    assert B.sp24_gemm_plan(128, 11008, 4096, B.SP24_BF16)["kernel"] == "splitk"
+    # the one-accumulator 256-token pair tile for the INT8 workload shape
+    assert B.sp24_gemm_plan(8192, 4096, 4096, B.SP24_INT8)["kernel"] == "pair256"
     monkeypatch.setenv("SP24_GEMM_IMPL", "pair240")
     forced = B.sp24_gemm_plan(4096, 3072, 768, B.SP24_BF16)
     assert forced["kernel"] == "pair240" and forced["tile_tokens"] == 240
