@@ -161,7 +161,9 @@ def test_conv3x3_large_batch_timing_and_parity():
 # k-blocks (the last half k-block reads past K), a last tile past the final
 # image (M = 192 < 256), and Cout not a multiple of the 256-channel pair tile
 IMPLICIT_BF16 = [(2, 8, 16, 64, 64), (4, 28, 28, 128, 128), (2, 56, 56, 64, 64),
-                 (3, 8, 8, 64, 256), (1, 16, 32, 128, 192)]
+                 (3, 8, 8, 64, 256), (1, 16, 32, 128, 192),
+                 # output channels that fill neither a 128-row nor a 256-row tile
+                 (2, 8, 32, 64, 72), (1, 16, 16, 128, 200)]
 
 
 @pytest.mark.parametrize("b,h,w,c,cout", IMPLICIT_BF16)
@@ -228,3 +230,30 @@ def test_implicit_conv3x3_rejects_untiled_shapes():
     # the automatic path falls back to the explicit gather for such shapes
     y = P.conv3x3(x, vals, meta, 64)
     assert y.shape == (1, 14, 14, 64) and B.sp24_device_status() == B.SP24_OK
+
+
+def test_implicit_conv3x3_int8_requantised_output():
+    # int8 codes in, int8 codes out (requantised with s_y), single-SM tiles
+    # with 4 boxes of 2 image rows per tile and a partial last tile
+    b, h, w, c, cout = 3, 10, 16, 128, 32
+    w4 = I.normal_bf16((cout, 3, 3, c), 0.02, 91)
+    x = I.normal_f32((b, h, w, c), 1.0, 92)
+    wflat = w4.view(cout, 9 * c).cuda()
+    mask = P.prune(wflat, B.SP24_MAGNITUDE, 2)
+    s_w = P.wscale(wflat, mask)
+    vals, meta = P.compress(wflat, mask, B.SP24_INT8, s_w)
+    xd = x.cuda()
+    s_x = P.act_scale(xd)
+    xq = P.quantize(xd, s_x)
+    s_y = torch.tensor([0.05], dtype=torch.float32, device="cuda")
+    y8 = P.conv3x3(xq, vals, meta, cout, dtype=B.SP24_INT8, s_x=s_x, s_w=s_w,
+                   out_kind=B.SP24_OUT_INT8, s_y=s_y, path="implicit")
+    assert B.sp24_device_status() == B.SP24_OK
+    wf = f64(w4.view(cout, 9 * c))
+    keep = O.prune(wf, O.MAGNITUDE, 2)
+    rs = O.channel_scales(wf, keep)
+    rv, rm = O.compress(O.quantize(wf, rs[:, None]), keep)
+    sx = O.tensor_scale(x.numpy().astype(np.float64))
+    acc = O.gemm_int8_acc(O.im2col3x3(O.quantize(x.numpy(), sx)), rv, rm, 9 * c)
+    ref = O.requant_int8(acc, sx, rs, np.float32(0.05))
+    assert np.array_equal(y8.cpu().numpy().reshape(-1, cout), ref)

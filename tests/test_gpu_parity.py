@@ -170,6 +170,24 @@ def test_prune_progressive_one_pass(mode, nkm):
         assert np.array_equal(ws[: 8 * k].view(torch.float64).cpu().numpy(), O.column_norms(f64(Xc)))
 
 
+def test_prune_progressive_then_int8_compress():
+    # the progressive masks feed the INT8 path: scales over the 2:4 mask, int8
+    # values and metadata bit for bit
+    w = I.int8_long_tail(M=16)
+    Wd = w.W.cuda()
+    m1, m2, _, _ = P.prune_progressive(Wd, B.SP24_MAGNITUDE, None, compress=False)
+    s_w = P.wscale(Wd, m2)
+    vals, meta = P.compress(Wd, m2, B.SP24_INT8, s_w)
+    ok_status()
+    r1, r2 = O.progressive(f64(w.W), O.MAGNITUDE)
+    assert np.array_equal(keep_of(m1, w.K), r1) and np.array_equal(keep_of(m2, w.K), r2)
+    rs = O.channel_scales(f64(w.W), r2)
+    assert np.array_equal(s_w.cpu().numpy(), rs)
+    rv, rm = O.compress(O.quantize(f64(w.W), rs[:, None]), r2)
+    assert np.array_equal(vals.cpu().numpy(), rv)
+    assert np.array_equal(canon_meta(meta, w.N, w.K, L.INT8), rm)
+
+
 def test_prune_llm_full():
     w = I.llm_proj(11008, 4096, 16)
     mask = P.prune(w.W.cuda(), B.SP24_MAGNITUDE, 2)
