@@ -181,7 +181,7 @@ class Runner:
     # number of library kernel launches per step (see the calls below)
     def launches_per_step(self) -> int:
         if self.wl.int8:
-            return 1 + 1 + 1 + 7 + 1 + 1     # prune, wscale, compress, act_scale, quantize, gemm
+            return 1 + 7 + 1 + 1             # weight conversion, act_scale, quantize, gemm
         if self.wanda:
             # the library forms the column norms inside the prune kernel when
             # row tiles x calibration rows is small, else launches colnorm first
@@ -198,13 +198,11 @@ class Runner:
         wl = self.wl
         rec(0)
         if wl.int8:
-            # (a second stream for the activation side was measured slower:
-            # its many small CTAs keep the weight-side persistent kernels off
-            # the SMs)
-            B.sp24_prune(self.W, None, B.SP24_MAGNITUDE, 2, None, self.mask2, None)
-            B.sp24_wscale(self.W, self.mask2, 0.9999, self.s_w)
+            # weight side: 2:4 mask, per-channel scale and int8 compression in
+            # one pass over W; activation side: per-tensor scale, quantisation
+            B.sp24_prune_compress_int8(self.W, 0.9999, self.mask2, self.s_w, self.vals,
+                                       self.meta)
             rec(1)
-            B.sp24_compress(self.W, self.mask2, B.SP24_INT8, self.s_w, self.vals, self.meta)
             B.sp24_act_scale(self.X, 0.9999, self.s_x, self.act_ws)
             B.sp24_quantize(self.X, self.s_x, self.Xq)
             rec(2)
@@ -246,12 +244,12 @@ class Runner:
 
     def compress_bytes(self) -> float:
         """Algorithmic bytes of the compression stage (fused prune+compress for
-        bf16: read W, write values + metadata)."""
-        N, K = self.N, self.K
+        bf16: read W, write values + metadata; INT8: the activation side)."""
+        N, K, M = self.N, self.K, self.M
         if self.wl.int8:
-            # compress int8: read W + mask, write values + metadata; the
-            # activation scale passes and quantisation share the stage
-            return 2 * N * K + N * K / 8 + N * K / 2 + N * K / 8
+            # activation scale (one pass over float32 X; the sample is
+            # negligible) and quantisation (read X, write Xq)
+            return 4 * M * K + 4 * M * K + M * K
         if self.wl.progressive:
             # one pass: read W (and Xc), write both masks, values and metadata
             mc = self.wl.Xc.shape[0] if self.wl.Xc is not None else 0
@@ -261,7 +259,9 @@ class Runner:
     def prune_bytes(self) -> float:
         N, K = self.N, self.K
         if self.wl.int8:
-            return 2 * N * K + N * K / 8 + (2 * N * K + N * K / 8 + 4 * N)   # prune + wscale
+            # one-pass weight conversion: read W, write mask, scales, int8
+            # values and metadata
+            return 2 * N * K + N * K / 8 + 4 * N + N * K / 2 + N * K / 8
         if self.wanda:
             mc = self.wl.Xc.shape[0]
             return 2 * mc * K + 8 * K + 2 * N * K + 8 * K + N * K / 8
@@ -506,6 +506,16 @@ def measure_config(name, device, flush, peaks, steps):
                            "frac_hbm": c_gbs / peaks["hbm_gbs"],
                            "prune_us": 1e3 * statistics.median(prune)},
     }
+    if wl.int8:
+        # INT8: the first stage is the one-pass weight conversion, the second
+        # the activation side (scale and quantisation)
+        prune_ms = statistics.median(prune)
+        p_gbs = runner.prune_bytes() / (prune_ms * 1e-3) / 1e9
+        out["prune_compress"]["stages"] = ("prune_us: weight conversion (mask, scales, int8 "
+                                           "compression); us: activation scale + quantisation")
+        out["prune_compress"]["prune_gbs"] = p_gbs
+        out["prune_compress"]["prune_frac_hbm"] = p_gbs / peaks["hbm_gbs"]
+        out["prune_compress"]["prep_us"] = 1e3 * (prune_ms + comp_ms)
     del runner
     torch.cuda.empty_cache()
     return out

@@ -257,6 +257,21 @@ sp24_status sp24_prune_compress(const void* W, int64_t N, int64_t K, int mode,
                                 uint8_t* mask_out, int dtype, const float* s_w,
                                 void* vals, void* meta, void* stream);
 
+/* INT8 weight conversion in one pass over W ([Ampere-sparsity] "PTQ and QAT"
+ * for the per-channel scale at `coverage`; [Orin ch.7] 2.1 Steps 1-2 for the
+ * magnitude 2:4 mask and the compressed stream): the outputs of
+ *   sp24_prune(W, mode = SP24_MAGNITUDE, n_keep = 2)          -> mask_out,
+ *   sp24_wscale(W, that mask, coverage)                      -> s_w,
+ *   sp24_compress(W, that mask, SP24_INT8, s_w)              -> vals, meta,
+ * bit for bit, from one kernel instead of three passes over W.
+ *   W: bf16 [N][K].  mask_out: sp24_mask_bytes(N, K) bytes or NULL.
+ *   s_w: float32 [N].  vals: int8 [N][K/2].  meta: sp24_meta_bytes(N, K).
+ * Rules: N >= 0, K >= 32, K % 32 == 0, 0 < coverage <= 1; W, vals and meta
+ * 16-byte aligned. */
+sp24_status sp24_prune_compress_int8(const void* W, int64_t N, int64_t K, double coverage,
+                                     uint8_t* mask_out, float* s_w, void* vals, void* meta,
+                                     void* stream);
+
 /* Progressive pruning in one pass ([Ampere-sparsity] Figure 4: the 25 %
  * stage keeps 3 of every 4 weights, the 50 % stage keeps 2 of 4 of the
  * weights the first stage kept).  With no fine-tuning between the stages both

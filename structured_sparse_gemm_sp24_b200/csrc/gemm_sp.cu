@@ -138,6 +138,7 @@ struct Plan {
   int impl;            // Impl
   int bn;              // split-K kernel: tokens per tile
   int split;           // split-K kernel: K slices (= cluster size)
+  bool small_ring;     // split-K kernel: the ring that lets several CTAs share an SM
   int64_t ctas;        // CTAs launched
   int cluster;         // CTAs per cluster
   int tile_tokens;     // tokens (rows of X and Y) per output tile
@@ -151,7 +152,33 @@ struct Plan {
 // all CTAs still fit one wave (SP24_SPLITK overrides the split).  Measured on
 // B200: M = 128 x 11008 x 4096 (86 tiles) takes 22.5 us split-K, 24.6 us on
 // the persistent kernel.
-sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
+// Split-K rings: the full ring (one CTA per SM) and a small one with which
+// several split CTAs share an SM (so that a split spreads a few row tiles
+// over every SM without a second wave).  Shared memory per SM on sm_100 is
+// 228 KiB, of which each resident CTA also takes 1 KiB.  With either ring
+// the CTAs that fit an SM by shared memory need at most 512 tensor-memory
+// columns together (16 tokens: 3 x 32; 32: 4 x 64; 64: 3 x 128; 128:
+// 2 x 256), so no CTA's allocation ever waits on another's.
+constexpr int kSmemPerSm = 228 * 1024;
+constexpr int small_ring_stages(int bn) { return bn == 16 ? 3 : 2; }
+
+template <int kDtype>
+int small_ring_smem(int bn) {
+  switch (bn) {
+    case 16: return GemmCfg<kDtype, 16, small_ring_stages(16)>::kSmemBytes;
+    case 32: return GemmCfg<kDtype, 32, small_ring_stages(32)>::kSmemBytes;
+    case 64: return GemmCfg<kDtype, 64, small_ring_stages(64)>::kSmemBytes;
+    default: return GemmCfg<kDtype, 128, small_ring_stages(128)>::kSmemBytes;
+  }
+}
+
+int small_ring_ctas_per_sm(int dtype, int bn) {
+  const int smem = dtype == SP24_BF16 ? small_ring_smem<SP24_BF16>(bn)
+                                      : small_ring_smem<SP24_INT8>(bn);
+  return kSmemPerSm / (smem + 1024);
+}
+
+sp24_status make_plan(int64_t m, int64_t n, int kblocks, int dtype, Plan* p) {
   const int sms = sm_count();
   const int64_t row_tiles = (n + 127) / 128;
   const int forced = impl_override();
@@ -178,6 +205,7 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
     p->impl = impl;
     p->bn = 128;
     p->split = 1;
+    p->small_ring = false;
     if (impl == kSingle) {
       const int64_t tiles = row_tiles * ((m + 127) / 128);
       p->ctas = tiles < sms ? tiles : sms;
@@ -196,18 +224,35 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
   }
   const int bn = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : 128;
   const int64_t base = row_tiles * ((m + bn - 1) / bn);
-  // one CTA per SM fits (the rings take most of shared memory), so the K
-  // split stops where the CTAs would exceed one wave: measured on B200 for
-  // M = 16..256 decode shapes, a second wave costs more than the longer K
-  // loop of a smaller split (e.g. M = 16, 11008 x 4096: split 1 on 86 SMs
-  // 20.5 us, split 4 on 344 CTAs 29 us)
+  // The split.  A stage's sparse MMAs take about the same time whatever the
+  // token count (measured on B200: ~0.44 us per 128-channel x 128-K stage at
+  // 16 tokens, ~0.5 us at 256), so at few tokens the kernel is bound by the
+  // stages the busiest SM runs: ceil(CTAs / SMs) x stages per CTA.  The plan
+  // takes the split (1, 2, 4, 8; at least 4 stages per CTA) that minimises
+  // it, the fewer CTAs on a tie, and stops before a second wave; more than
+  // one CTA per SM takes the small ring.  E.g. M = 16, 11008 x 4096 (86 row
+  // tiles, 32 stages): split 1 on 86 SMs runs 32 stages on the busiest SM,
+  // split 4 (344 CTAs, 3 per SM) 24 -- 9.8 against 14.3 us a launch,
+  // measured back to back.
   int split = 1;
-  while (split < 8 && base * split * 2 <= sms && kblocks >= 4 * split) split *= 2;
+  int64_t best = -1;
+  const int cap = small_ring_ctas_per_sm(dtype, bn);
+  for (int sp = 1; sp <= 8; sp *= 2) {
+    if (sp > 1 && kblocks < 4 * sp) break;
+    const int64_t per_sm = (base * sp + sms - 1) / sms;
+    if (sp > 1 && per_sm > cap) break;
+    const int64_t cost = per_sm * ((kblocks + sp - 1) / sp);
+    if (best < 0 || cost < best) {
+      best = cost;
+      split = sp;
+    }
+  }
   const int so = split_override();
   if (so > 0 && so <= kblocks) split = so;
   p->impl = kSplitK;
   p->bn = bn;
   p->split = split;
+  p->small_ring = base * split > sms;
   p->ctas = base * split;
   p->cluster = split;
   p->tile_tokens = bn;
@@ -218,7 +263,7 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, Plan* p) {
 template <int kDtype>
 sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s) {
   Plan p;
-  SP24_TRY(make_plan(a.m, a.n, a.kblocks, &p));
+  SP24_TRY(make_plan(a.m, a.n, a.kblocks, kDtype, &p));
   a.kb_per_split = (a.kblocks + p.split - 1) / p.split;
   const int bn = p.bn;
   const int el = kDtype == SP24_BF16 ? 2 : 1;
@@ -261,6 +306,15 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
 
 #define SP24_GEMM_CASE(BN_, ST_)                                                          \
   if (bn == BN_) {                                                                        \
+    constexpr int kSm = small_ring_stages(BN_);                                           \
+    if (p.small_ring) {                                                                   \
+      switch (split) {                                                                    \
+        case 1: return launch_gemm_cfg<kDtype, BN_, kSm, 1>(ma, mb, a, s);                \
+        case 2: return launch_gemm_cfg<kDtype, BN_, kSm, 2>(ma, mb, a, s);                \
+        case 4: return launch_gemm_cfg<kDtype, BN_, kSm, 4>(ma, mb, a, s);                \
+        default: return launch_gemm_cfg<kDtype, BN_, kSm, 8>(ma, mb, a, s);               \
+      }                                                                                   \
+    }                                                                                     \
     switch (split) {                                                                      \
       case 1: return launch_gemm_cfg<kDtype, BN_, ST_, 1>(ma, mb, a, s);                  \
       case 2: return launch_gemm_cfg<kDtype, BN_, ST_, 2>(ma, mb, a, s);                  \
@@ -329,7 +383,7 @@ extern "C" sp24_status sp24_gemm_plan(int64_t M, int64_t N, int64_t K, int dtype
   SP24_TRY(check_device());
   const int kl = dtype == SP24_BF16 ? 128 : 256;
   Plan p;
-  SP24_TRY(make_plan(M, N, static_cast<int>((K + kl - 1) / kl), &p));
+  SP24_TRY(make_plan(M, N, static_cast<int>((K + kl - 1) / kl), dtype, &p));
   std::memset(plan, 0, sizeof(*plan));
   std::snprintf(plan->kernel, sizeof(plan->kernel), "%s", impl_name(p.impl));
   plan->tile_tokens = p.tile_tokens;

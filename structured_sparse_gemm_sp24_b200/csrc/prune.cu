@@ -1181,6 +1181,176 @@ __global__ void __launch_bounds__(256) fake_quant_kernel(const uint4* __restrict
   }
 }
 
+// ------------------------------------ a2..a5 INT8 weight conversion, one pass
+// Magnitude 2:4 pruning, the per-row weight scale and the int8 compression of
+// W in one kernel: the outputs of sp24_prune (n_keep = 2), sp24_wscale and
+// sp24_compress(SP24_INT8) without their three passes over W.  One warp per
+// row (8 rows per 256-thread block):
+//  * pass 1 reads the row and takes its largest |w| key.  The largest
+//    magnitude of a group is always kept, so this is the largest kept key;
+//    every group keeps exactly two positions, so the kept count c = K/2 and
+//    the nearest rank r = max(1, ceil(coverage * c)) are known up front.  When
+//    r = c the scale is that maximum; otherwise the weight-scale kernel's two
+//    histogram passes over the kept keys select the r-th smallest;
+//  * pass 2 reads the row again (its bytes are still in L2) and writes the
+//    keep mask, the int8 values (q8, the quantiser of sp24_compress) and the
+//    metadata bytes.  Positions >= K up to the 128-position chunk and rows
+//    >= N up to the 128-row tile get the padding pattern (0, 1), as
+//    sp24_compress writes them.
+template <class F>
+__device__ __forceinline__ void for_kept_keys(const uint4* wr, int64_t kvec, uint32_t lane, F&& f) {
+  for (int64_t v = lane; v < kvec; v += 32) {
+    const uint4 q = __ldg(wr + v);
+    uint32_t lo0, hi0, lo1, hi1;
+    top2_positions_mag<false>(q.x, q.y, 0xFu, lo0, hi0);
+    top2_positions_mag<false>(q.z, q.w, 0xFu, lo1, hi1);
+    const uint32_t p0 = gather_pair(q.x, q.y, lo0, hi0);
+    const uint32_t p1 = gather_pair(q.z, q.w, lo1, hi1);
+    f(mag_key(p0));
+    f(mag_key(p0 >> 16));
+    f(mag_key(p1));
+    f(mag_key(p1 >> 16));
+  }
+}
+
+// Writes the outputs of one row's vector v (8 weights) given the row scale.
+__device__ __forceinline__ void int8_emit(const uint4& q, int64_t v, float s, float rs,
+                                          uint32_t* vr, uint8_t* mr, uint8_t* mrow) {
+  uint32_t lo0, hi0, lo1, hi1;
+  top2_positions_mag<false>(q.x, q.y, 0xFu, lo0, hi0);
+  top2_positions_mag<false>(q.z, q.w, 0xFu, lo1, hi1);
+  const uint32_t p0 = gather_pair(q.x, q.y, lo0, hi0);
+  const uint32_t p1 = gather_pair(q.z, q.w, lo1, hi1);
+  const uint32_t packed = q8(__uint_as_float(p0 << 16), s, rs) |
+                          (q8(__uint_as_float(p0 & 0xFFFF0000u), s, rs) << 8) |
+                          (q8(__uint_as_float(p1 << 16), s, rs) << 16) |
+                          (q8(__uint_as_float(p1 & 0xFFFF0000u), s, rs) << 24);
+  __stcs(vr + v, packed);
+  if (mr) mr[v] = static_cast<uint8_t>((1u << lo0) | (1u << hi0) | (((1u << lo1) | (1u << hi1)) << 4));
+  mrow[(v >> 4) * 2048 + (v & 15)] = static_cast<uint8_t>(lo0 | (hi0 << 2) | (lo1 << 4) | (hi1 << 6));
+}
+
+__device__ __forceinline__ uint32_t vec_max_key(const uint4& q) {
+  const uint32_t m0 = max(mag_key(q.x), mag_key(q.x >> 16));
+  const uint32_t m1 = max(mag_key(q.y), mag_key(q.y >> 16));
+  const uint32_t m2 = max(mag_key(q.z), mag_key(q.z >> 16));
+  const uint32_t m3 = max(mag_key(q.w), mag_key(q.w >> 16));
+  return max(max(m0, m1), max(m2, m3));
+}
+
+// The r-th smallest kept key of a row (r < kept count): two histogram passes
+// over the kept keys, as the weight-scale kernel.
+__device__ __forceinline__ uint32_t int8_select_key(const uint4* wr, int64_t kvec, uint32_t r,
+                                                    uint32_t* h, uint32_t lane) {
+  for (uint32_t i = lane; i < 256; i += 32) h[i] = 0;
+  __syncwarp();
+  for_kept_keys(wr, kvec, lane, [&](uint32_t kk) { atomicAdd(&h[kk >> 7], 1u); });
+  __syncwarp();
+  uint32_t below = 0;
+  const uint32_t bucket = warp_find_bin(h, 256, r, below);
+  const uint32_t r2 = r - below;
+  __syncwarp();
+  for (uint32_t i = lane; i < 256; i += 32) h[i] = 0;
+  __syncwarp();
+  for_kept_keys(wr, kvec, lane, [&](uint32_t kk) {
+    if ((kk >> 7) == bucket) atomicAdd(&h[kk & 0x7Fu], 1u);
+  });
+  __syncwarp();
+  uint32_t below2 = 0;
+  return (bucket << 7) | warp_find_bin(h, 128, r2, below2);
+}
+
+// kRegVec > 0: the row (at most 32 * kRegVec vectors) stays in registers
+// between the passes, all its loads in flight at once; 0: any K, the row is
+// read in batches of 8 vectors per lane and again for the second pass.
+constexpr int kInt8RegVec = 16;   // rows up to K = 4096 in registers
+
+template <int kRegVec>
+__global__ void __launch_bounds__(256) prune_int8_kernel(const uint16_t* __restrict__ w, int64_t n,
+                                                         int64_t k, double coverage,
+                                                         uint8_t* __restrict__ mask_out,
+                                                         float* __restrict__ s_w,
+                                                         uint32_t* __restrict__ vals,
+                                                         uint8_t* __restrict__ meta) {
+  pdl_launch_dependents();
+  pdl_wait_prior();
+  __shared__ uint32_t hist[8][256];
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t wid = threadIdx.x >> 5;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + wid;
+  const int64_t kvec = k / 8;
+  const int kblocks = static_cast<int>((k + 127) / 128);
+  const int64_t kvec_pad = static_cast<int64_t>(kblocks) * 16;
+  // metadata of this row: chunk kb at + kb * 2048, vector bb of the chunk at + bb
+  uint8_t* mrow = meta + (row >> 7) * kblocks * 2048 + 16 * (row & 127);
+  if (row >= n) {   // a padding row of the last 128-row tile
+    for (int64_t v = lane; v < kvec_pad; v += 32) mrow[(v >> 4) * 2048 + (v & 15)] = 0x44u;
+    return;
+  }
+  const uint4* wr = reinterpret_cast<const uint4*>(w + row * k);
+  uint4 reg[kRegVec > 0 ? kRegVec : 1];
+  uint32_t kmax = 0;
+  if constexpr (kRegVec > 0) {
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i) {
+      const int64_t v = lane + 32 * i;
+      reg[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i) kmax = max(kmax, vec_max_key(reg[i]));
+  } else {
+    for (int64_t v0 = lane; v0 < kvec; v0 += 32 * 8) {
+      uint4 b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t v = v0 + 32 * i;
+        b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) kmax = max(kmax, vec_max_key(b[i]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+  const uint32_t cnt = static_cast<uint32_t>(kvec * 4);
+  uint32_t key = kmax;
+  {
+    const double rd = ceil(coverage * static_cast<double>(cnt));
+    uint32_t r = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
+    if (r > cnt) r = cnt;
+    if (r < cnt) key = int8_select_key(wr, kvec, r, hist[wid], lane);
+  }
+  const float t = __uint_as_float(key << 16);
+  const float s = (cnt == 0 || t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
+  if (lane == 0) s_w[row] = s;
+  const float rs = __frcp_rn(s);
+  uint8_t* mr = mask_out ? mask_out + row * kvec : nullptr;
+  uint32_t* vr = vals + row * kvec;
+  if constexpr (kRegVec > 0) {
+#pragma unroll
+    for (int i = 0; i < kRegVec; ++i) {
+      const int64_t v = lane + 32 * i;
+      if (v < kvec) int8_emit(reg[i], v, s, rs, vr, mr, mrow);
+    }
+  } else {
+    for (int64_t v0 = lane; v0 < kvec; v0 += 32 * 8) {
+      uint4 b[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t v = v0 + 32 * i;
+        b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int64_t v = v0 + 32 * i;
+        if (v < kvec) int8_emit(b[i], v, s, rs, vr, mr, mrow);
+      }
+    }
+  }
+  // positions >= K of the last 128-position chunk: the padding pattern
+  for (int64_t v = kvec + lane; v < kvec_pad; v += 32) mrow[(v >> 4) * 2048 + (v & 15)] = 0x44u;
+}
+
 // ------------------------------------------- Wanda prune without allocation
 // For callers that may not allocate device memory (see sp24_prune_wanda_noalloc
 // in include/sp24.h): the float64 column norms live in this file-scope array
@@ -1520,6 +1690,27 @@ sp24_status sp24_fake_quant(const void* W, const uint8_t* mask, int64_t N, int64
   return launch_kernel(fake_quant_kernel, dim3(gx, gy), dim3(256), 0, as_stream(stream), 1,
                        static_cast<const uint4*>(W), mask, s_w, N, kvec,
                        static_cast<uint4*>(W_fq));
+}
+
+sp24_status sp24_prune_compress_int8(const void* W, int64_t N, int64_t K, double coverage,
+                                    uint8_t* mask_out, float* s_w, void* vals, void* meta,
+                                    void* stream) {
+  if (N < 0 || K < 0 || !(coverage > 0.0 && coverage <= 1.0)) return SP24_ERR_ARG;
+  if (K < 32 || K % 32 != 0) return SP24_ERR_ALIGN;
+  if (N == 0) return SP24_OK;
+  if (!W || !s_w || !vals || !meta) return SP24_ERR_ARG;
+  if (!aligned16(W) || !aligned16(vals) || !aligned16(meta)) return SP24_ERR_ALIGN;
+  if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return SP24_ERR_UNSUPPORTED;
+  SP24_TRY(check_device());
+  const int64_t n_pad = (N + 127) / 128 * 128;   // padding rows of the last tile too
+  const dim3 grid(static_cast<unsigned>(n_pad / 8));
+  if (K / 8 <= 32 * kInt8RegVec)
+    return launch_kernel(prune_int8_kernel<kInt8RegVec>, grid, dim3(256), 0, as_stream(stream),
+                         1, static_cast<const uint16_t*>(W), N, K, coverage, mask_out, s_w,
+                         static_cast<uint32_t*>(vals), static_cast<uint8_t*>(meta));
+  return launch_kernel(prune_int8_kernel<0>, grid, dim3(256), 0, as_stream(stream), 1,
+                       static_cast<const uint16_t*>(W), N, K, coverage, mask_out, s_w,
+                       static_cast<uint32_t*>(vals), static_cast<uint8_t*>(meta));
 }
 
 sp24_status sp24_quantize(const float* X, int64_t count, const float* s_x, int8_t* Xq,

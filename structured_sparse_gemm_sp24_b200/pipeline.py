@@ -85,6 +85,17 @@ def prune_compress(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE,
     return (vals, meta, mask) if want_mask else (vals, meta)
 
 
+def prune_compress_int8(W: torch.Tensor, coverage: float = COVERAGE, want_mask: bool = False):
+    """INT8 weight conversion in one pass: (vals int8, meta, s_w[, mask]) as
+    prune (magnitude, 2 of 4) -> wscale -> compress(SP24_INT8) give them."""
+    N, K = W.shape
+    vals, meta = alloc_compressed(N, K, _b.SP24_INT8, W.device)
+    s_w = torch.empty(N, dtype=torch.float32, device=W.device)
+    mask = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device) if want_mask else None
+    _b.sp24_prune_compress_int8(W, coverage, mask, s_w, vals, meta)
+    return (vals, meta, s_w, mask) if want_mask else (vals, meta, s_w)
+
+
 def prune_progressive(W: torch.Tensor, mode: int = _b.SP24_MAGNITUDE,
                       Xc: Optional[torch.Tensor] = None, compress: bool = True):
     """Progressive pruning in one pass: (mask1 keeping 3 of 4, mask2 keeping 2 of

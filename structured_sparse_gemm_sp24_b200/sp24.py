@@ -58,6 +58,8 @@ SIGNATURES = {
     "sp24_compress": (_c_int, [_c_p, _c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p, _c_p]),
     "sp24_prune_compress": (_c_int, [_c_p, _c_i64, _c_i64, _c_int, _c_p, _c_p, _c_p, _c_int,
                                      _c_p, _c_p, _c_p, _c_p]),
+    "sp24_prune_compress_int8": (_c_int, [_c_p, _c_i64, _c_i64, _c_dbl, _c_p, _c_p, _c_p, _c_p,
+                                          _c_p]),
     "sp24_prune_progressive": (_c_int, [_c_p, _c_i64, _c_i64, _c_p, _c_i64, _c_int, _c_p, _c_p,
                                         _c_p, _c_p, _c_p, _c_p]),
     "sp24_conv3x3": (_c_int, [_c_p, _c_i64, _c_i64, _c_i64, _c_i64, _c_p, _c_p, _c_i64, _c_int,
@@ -252,6 +254,15 @@ def sp24_prune_progressive(W: torch.Tensor, Xc: Optional[torch.Tensor], mode: in
     _check(lib().sp24_prune_progressive(_ptr(W), N, K, _ptr(Xc), Mc, mode, _ptr(mask1_out),
                                         _ptr(mask2_out), _ptr(vals), _ptr(meta), _ptr(workspace),
                                         _stream(stream)), "sp24_prune_progressive")
+
+
+def sp24_prune_compress_int8(W: torch.Tensor, coverage: float, mask_out: Optional[torch.Tensor],
+                             s_w: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor,
+                             stream=None) -> None:
+    N, K = W.shape
+    _check(lib().sp24_prune_compress_int8(_ptr(W), N, K, coverage, _ptr(mask_out), _ptr(s_w),
+                                          _ptr(vals), _ptr(meta), _stream(stream)),
+           "sp24_prune_compress_int8")
 
 
 def sp24_conv3x3(X: torch.Tensor, vals: torch.Tensor, meta: torch.Tensor, Cout: int, dtype: int,

@@ -123,6 +123,19 @@ def test_compress_and_gemm_host_validation(lib):
              None, None) == B.SP24_OK
 
 
+def test_prune_compress_int8_host_validation(lib):
+    f = lib.sp24_prune_compress_int8
+    args = lambda n, k, cov, w=FAKE: (w, n, k, ctypes.c_double(cov), None, FAKE, FAKE, FAKE, None)
+    assert f(*args(8, 48, 0.9999)) == B.SP24_ERR_ALIGN        # K % 32
+    assert f(*args(8, 16, 0.9999)) == B.SP24_ERR_ALIGN        # K < 32
+    assert f(*args(8, 64, 0.0)) == B.SP24_ERR_ARG             # coverage outside (0, 1]
+    assert f(*args(8, 64, 1.5)) == B.SP24_ERR_ARG
+    assert f(*args(-1, 64, 0.9999)) == B.SP24_ERR_ARG
+    assert f(*args(8, 64, 0.9999, w=FAKE + 4)) == B.SP24_ERR_ALIGN
+    assert f(FAKE, 8, 64, ctypes.c_double(0.9999), None, None, FAKE, FAKE, None) == B.SP24_ERR_ARG
+    assert f(*args(0, 64, 0.9999, w=None)) == B.SP24_OK      # empty: a no-op
+
+
 def test_scale_host_validation(lib):
     assert lib.sp24_wscale(FAKE, FAKE, 8, 16, 0.0, FAKE, None) == B.SP24_ERR_ARG
     assert lib.sp24_wscale(FAKE, FAKE, 8, 16, 1.5, FAKE, None) == B.SP24_ERR_ARG

@@ -232,6 +232,36 @@ def test_compress_int8(shape):
     ok_status()
 
 
+@pytest.mark.parametrize("case", [("int8_workload", 0.9999), ((130, 256), 0.5), ((1, 32), 0.9999),
+                                  ((200, 4128), 0.9999), ((257, 1056), 0.9), ((64, 512), 1.0)])
+def test_prune_compress_int8_one_pass(case):
+    # the one-pass INT8 weight conversion against the three kernels it
+    # replaces (every byte, metadata padding included) and the oracle
+    shape, cov = case
+    if shape == "int8_workload":
+        w = I.int8_long_tail().W                      # 4096 x 4096, 1 % long tail
+    else:
+        w = I.long_tail_bf16(shape, 0.02, seed=5, tail_seed=8)
+    n, k = w.shape
+    wd = w.cuda()
+    vals, meta, s_w, mask = P.prune_compress_int8(wd, cov, want_mask=True)
+    ok_status()
+    m3 = P.prune(wd, B.SP24_MAGNITUDE, 2)
+    s3 = P.wscale(wd, m3, cov)
+    v3, t3 = P.compress(wd, m3, B.SP24_INT8, s3)
+    assert torch.equal(mask, m3) and torch.equal(s_w, s3)
+    assert torch.equal(vals, v3) and torch.equal(meta, t3)
+    keep = O.prune(f64(w), O.MAGNITUDE, 2)
+    rs = O.channel_scales(f64(w), keep, cov)
+    assert np.array_equal(keep_of(mask, k), keep)
+    assert np.array_equal(s_w.cpu().numpy(), rs)
+    rv, rm = O.compress(O.quantize(f64(w), rs[:, None]), keep)
+    assert np.array_equal(vals.cpu().numpy(), rv)
+    assert np.array_equal(canon_meta(meta, n, k, L.INT8), rm)
+    assert L.padding_is_valid(meta.cpu().numpy(), n, k, L.INT8)
+    ok_status()
+
+
 @pytest.mark.parametrize("dtype", [B.SP24_BF16, B.SP24_INT8])
 @pytest.mark.parametrize("mode", [B.SP24_MAGNITUDE, B.SP24_WANDA])
 def test_prune_compress_fused(mode, dtype):
@@ -464,10 +494,11 @@ def test_gemm_bf16_square_sampled_large(n):
 
 
 def test_gemm_bf16_deterministic_split():
-    w = I.llm_proj(4096, 11008, 16)      # split-K over a cluster
-    _, vals, meta, y1 = _bf16_pipeline(w.W, w.X)
-    y2 = P.gemm(w.X.cuda(), vals, meta, w.N)
-    assert torch.equal(y1, y2)
+    for n, k in [(4096, 11008), (11008, 4096)]:     # split-K over a cluster (the second
+        w = I.llm_proj(n, k, 16)                    # with CTAs sharing SMs)
+        _, vals, meta, y1 = _bf16_pipeline(w.W, w.X)
+        y2 = P.gemm(w.X.cuda(), vals, meta, w.N)
+        assert torch.equal(y1, y2)
 
 
 def test_gemm_empty_is_noop():
@@ -621,6 +652,38 @@ def test_gemm_splitk_forced(split, mnk, monkeypatch):
     ok_status()
 
 
+# --------------------------------------------- split-K with CTAs sharing SMs
+@pytest.mark.parametrize("mnk", [(16, 11008, 4096), (64, 11008, 4096), (40, 11008, 2048 + 96)])
+def test_gemm_splitk_small_ring(mnk, monkeypatch):
+    # more split CTAs than SMs (several per SM on the small ring): bf16 within
+    # the bound, int8 accumulators exact
+    monkeypatch.delenv("SP24_GEMM_IMPL", raising=False)
+    monkeypatch.delenv("SP24_SPLITK", raising=False)
+    m, n, k = mnk
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = B.sp24_gemm_plan(m, n, k, B.SP24_BF16)
+    assert plan["kernel"] == "splitk" and plan["split_k"] > 1 and plan["ctas"] > sms
+    W = I.normal_bf16((n, k), 1.0, seed=66)
+    X = I.normal_bf16((m, k), 1.0, seed=67)
+    Wd = W.cuda()
+    vals, meta = P.compress(Wd, P.prune(Wd, B.SP24_MAGNITUDE, 2), B.SP24_BF16)
+    y = P.gemm(X.cuda(), vals, meta, n)
+    ok_status()
+    assert_bf16_close(y, *_bf16_ref(W, X))
+    Wi = I.long_tail_bf16((n, k), 0.02, seed=68, tail_seed=69)
+    Xi = I.normal_f32((m, k), 1.0, seed=70)
+    acc, _, _ = _int8_ref(Wi, Xi)
+    Wid = Wi.cuda()
+    mask = P.prune(Wid, B.SP24_MAGNITUDE, 2)
+    gw = P.wscale(Wid, mask)
+    vq, mq = P.compress(Wid, mask, B.SP24_INT8, gw)
+    xd = Xi.cuda()
+    gx = P.act_scale(xd)
+    y32 = P.gemm(P.quantize(xd, gx), vq, mq, n, B.SP24_INT8, gx, gw, B.SP24_OUT_INT32)
+    ok_status()
+    assert np.array_equal(y32.cpu().numpy(), acc)
+
+
 # ------------------------------------------------------ Sparse-QAT fake quant
 @pytest.mark.parametrize("case", ["int8_workload", "ragged_3of4"])
 def test_fake_quant_matches_oracle(case):
@@ -724,6 +787,13 @@ def test_gemm_plan_families(monkeypatch):
     assert conv["kernel"] == "single" and conv["ctas"] == sms
     # less than one wave of 128 x 128 tiles (86 for N = 11008): split-K
     assert B.sp24_gemm_plan(128, 11008, 4096, B.SP24_BF16)["kernel"] == "splitk"
+    # 16 tokens, 86 row tiles of 32 stages: split 4 with three CTAs per SM
+    # (24 stages on the busiest SM against 32 unsplit)
+    dec = B.sp24_gemm_plan(16, 11008, 4096, B.SP24_BF16)
+    assert dec["split_k"] == 4 and dec["ctas"] == 344
+    # 32 row tiles of 86 stages: split 4, one CTA per SM
+    dec2 = B.sp24_gemm_plan(16, 4096, 11008, B.SP24_BF16)
+    assert dec2["split_k"] == 4 and dec2["ctas"] == 128
     # the one-accumulator 256-token pair tile for the INT8 workload shape
     assert B.sp24_gemm_plan(8192, 4096, 4096, B.SP24_INT8)["kernel"] == "pair256"
     monkeypatch.setenv("SP24_GEMM_IMPL", "pair240")
