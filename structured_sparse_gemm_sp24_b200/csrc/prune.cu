@@ -330,15 +330,15 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     const int rt = c / a.kblocks, kb = c - rt * a.kblocks;
     const int st = i % kStreamStages;
     const uint8_t* sb = smem + st * kStreamStage;
-    const bool ready = mbar_wait(&full[st], (i / kStreamStages) & 1u);
     const int64_t kv = static_cast<int64_t>(kb) * 16 + bb;
-    const bool kv_ok = kv < kvec && ready;
     uint8_t* mb = meta_buf + (i & 1) * 2048;
     uint8_t* ob = mout_buf + (i & 1) * 2048;
     uint8_t* ob1 = mout1_buf + (i & 1) * 2048;
     double nrm[8];
     if constexpr (kWanda) {
       if (fused_norms) {
+        // (formed before waiting for the chunk: they need only Xc, so its
+        // loads overlap the W chunk's TMA)
         // column norms of this chunk, in the stage's norm slot (TMA does not
         // write it in this mode): Xc is staged 128 tokens at a time with
         // every 16-byte load in flight; threads 0..127 then add the squares
@@ -382,6 +382,10 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
         }
         __syncthreads();
       }
+    }
+    const bool ready = mbar_wait(&full[st], (i / kStreamStages) & 1u);
+    const bool kv_ok = kv < kvec && ready;
+    if constexpr (kWanda) {
 #pragma unroll
       for (int e = 0; e < 8; ++e)
         nrm[e] = reinterpret_cast<const double*>(sb + kWTile + kMTile)[bb * 8 + e];
