@@ -206,8 +206,7 @@ class Runner:
             B.sp24_act_scale(self.X, 0.9999, self.s_x, self.act_ws)
             B.sp24_quantize(self.X, self.s_x, self.Xq)
             rec(2)
-            B.sp24_gemm(self.Xq, self.vals, self.meta, self.N, B.SP24_INT8, self.s_x, self.s_w,
-                        B.SP24_OUT_BF16, None, self.Y)
+            self.gemm_call()
         elif self.wanda and wl.progressive:
             # one pass: norms, the 3:4 mask, the 2:4 mask on the survivors and
             # the compressed operand
@@ -215,8 +214,7 @@ class Runner:
             B.sp24_prune_progressive(self.W, self.Xc, B.SP24_WANDA, self.mask1, self.mask2,
                                      self.vals, self.meta, self.ws)
             rec(2)
-            B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
-                        B.SP24_OUT_BF16, None, self.Y)
+            self.gemm_call()
         elif self.wanda:
             # prune also leaves the float64 column norms in its workspace
             n_keep = 2
@@ -225,16 +223,23 @@ class Runner:
             B.sp24_prune_compress(self.W, B.SP24_WANDA, self.ws, None, None, B.SP24_BF16,
                                   None, self.vals, self.meta)
             rec(2)
-            B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
-                        B.SP24_OUT_BF16, None, self.Y)
+            self.gemm_call()
         else:
             rec(1)
             B.sp24_prune_compress(self.W, B.SP24_MAGNITUDE, None, None, None, B.SP24_BF16, None,
                                   self.vals, self.meta)
             rec(2)
+            self.gemm_call()
+        rec(3)
+
+    def gemm_call(self):
+        """The step's GEMM (its operands are the step's earlier outputs)."""
+        if self.wl.int8:
+            B.sp24_gemm(self.Xq, self.vals, self.meta, self.N, B.SP24_INT8, self.s_x, self.s_w,
+                        B.SP24_OUT_BF16, None, self.Y)
+        else:
             B.sp24_gemm(self.X, self.vals, self.meta, self.N, B.SP24_BF16, None, None,
                         B.SP24_OUT_BF16, None, self.Y)
-        rec(3)
 
     def flops(self) -> float:
         return 2.0 * self.M * self.N * self.K
@@ -485,6 +490,10 @@ def measure_config(name, device, flush, peaks, steps):
         runner.step()
     torch.cuda.synchronize()
     tot, prune, comp, gemm = time_steps(runner, steps, flush)
+    # the GEMM again, five launches back to back in one graph (per launch):
+    # how it runs between other kernels of a model, without the event nodes
+    # of the stage timing
+    b2b_ms = time_graph(lambda: [runner.gemm_call() for _ in range(5)], flush) / 5
     if B.sp24_device_status() != B.SP24_OK:
         raise SystemExit(f"device status not OK after config {name}")
     gemm_ms, comp_ms = statistics.median(gemm), statistics.median(comp)
@@ -501,7 +510,10 @@ def measure_config(name, device, flush, peaks, steps):
                  "bound": roof["bound"], "frac": roof["frac"],
                  "frac_of": ("sparse tensor peak" if roof["bound"] == "tensor" else "HBM") +
                             " (measured burst)",
-                 "traffic": gemm_traffic(wl.name, plan["kernel"])},
+                 "traffic": gemm_traffic(wl.name, plan["kernel"]),
+                 "back_to_back_us": 1e3 * b2b_ms,
+                 "frac_back_to_back": roofline_entry(runner, b2b_ms, peaks,
+                                                     sustained=False)["frac"]},
         "prune_compress": {"us": 1e3 * comp_ms, "gbs": c_gbs,
                            "frac_hbm": c_gbs / peaks["hbm_gbs"],
                            "prune_us": 1e3 * statistics.median(prune)},

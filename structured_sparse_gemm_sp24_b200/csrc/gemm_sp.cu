@@ -80,13 +80,13 @@ int impl_override() {
   return -1;
 }
 
-// SP24_SPLITK = 1 | 2 | 4 | 8: K slices of the split-K kernel (tuning
-// override; 0 = choose by shape).
+// SP24_SPLITK = 1..8: K slices of the split-K kernel (tuning override; 0 =
+// choose by shape).
 int split_override() {
   const char* e = std::getenv("SP24_SPLITK");
   if (!e) return 0;
   const int v = std::atoi(e);
-  return (v == 1 || v == 2 || v == 4 || v == 8) ? v : 0;
+  return (v >= 1 && v <= 8) ? v : 0;
 }
 
 const char* impl_name(int impl) {
@@ -228,12 +228,15 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, int dtype, Plan* p) {
   // token count (measured on B200: ~0.44 us per 128-channel x 128-K stage at
   // 16 tokens, ~0.5 us at 256), so at few tokens the kernel is bound by the
   // stages the busiest SM runs: ceil(CTAs / SMs) x stages per CTA.  The plan
-  // takes the split (1, 2, 4, 8; at least 4 stages per CTA) that minimises
-  // it, the fewer CTAs on a tie, and stops before a second wave; more than
-  // one CTA per SM takes the small ring.  E.g. M = 16, 11008 x 4096 (86 row
-  // tiles, 32 stages): split 1 on 86 SMs runs 32 stages on the busiest SM,
-  // split 4 (344 CTAs, 3 per SM) 24 -- 9.8 against 14.3 us a launch,
-  // measured back to back.
+  // takes the split among 1, 2, 4, 8 (at least 4 stages per CTA) that
+  // minimises it, the fewer CTAs on a tie; more than one CTA per SM takes
+  // the small ring.  E.g. M = 16, 11008 x 4096 (86 row tiles, 32 stages):
+  // split 1 on 86 SMs runs 32 stages on the busiest SM, split 4 (344 CTAs,
+  // 3 per SM) 24 -- 9.8 against 13.9 us a launch back to back.  Splits of 3,
+  // 5, 6 and 7 run correctly (SP24_SPLITK) but measured no better: at 3 CTAs
+  // per SM a GPC holds fewer 5-CTA clusters than the 86 tiles need
+  // (cudaOccupancyMaxActiveClusters: 82), and the second wave costs more
+  // than the shorter K loop saves.
   int split = 1;
   int64_t best = -1;
   const int cap = small_ring_ctas_per_sm(dtype, bn);
@@ -258,6 +261,21 @@ sp24_status make_plan(int64_t m, int64_t n, int kblocks, int dtype, Plan* p) {
   p->tile_tokens = bn;
   p->tile_channels = 128;
   return SP24_OK;
+}
+
+template <int kDtype, int BN, int ST>
+sp24_status launch_split(int split, const CUtensorMap& ma, const CUtensorMap& mb,
+                         const GemmArgs& a, cudaStream_t s) {
+  switch (split) {
+    case 1: return launch_gemm_cfg<kDtype, BN, ST, 1>(ma, mb, a, s);
+    case 2: return launch_gemm_cfg<kDtype, BN, ST, 2>(ma, mb, a, s);
+    case 3: return launch_gemm_cfg<kDtype, BN, ST, 3>(ma, mb, a, s);
+    case 4: return launch_gemm_cfg<kDtype, BN, ST, 4>(ma, mb, a, s);
+    case 5: return launch_gemm_cfg<kDtype, BN, ST, 5>(ma, mb, a, s);
+    case 6: return launch_gemm_cfg<kDtype, BN, ST, 6>(ma, mb, a, s);
+    case 7: return launch_gemm_cfg<kDtype, BN, ST, 7>(ma, mb, a, s);
+    default: return launch_gemm_cfg<kDtype, BN, ST, 8>(ma, mb, a, s);
+  }
 }
 
 template <int kDtype>
@@ -307,20 +325,8 @@ sp24_status dispatch(const void* x, const void* vals, GemmArgs a, cudaStream_t s
 #define SP24_GEMM_CASE(BN_, ST_)                                                          \
   if (bn == BN_) {                                                                        \
     constexpr int kSm = small_ring_stages(BN_);                                           \
-    if (p.small_ring) {                                                                   \
-      switch (split) {                                                                    \
-        case 1: return launch_gemm_cfg<kDtype, BN_, kSm, 1>(ma, mb, a, s);                \
-        case 2: return launch_gemm_cfg<kDtype, BN_, kSm, 2>(ma, mb, a, s);                \
-        case 4: return launch_gemm_cfg<kDtype, BN_, kSm, 4>(ma, mb, a, s);                \
-        default: return launch_gemm_cfg<kDtype, BN_, kSm, 8>(ma, mb, a, s);               \
-      }                                                                                   \
-    }                                                                                     \
-    switch (split) {                                                                      \
-      case 1: return launch_gemm_cfg<kDtype, BN_, ST_, 1>(ma, mb, a, s);                  \
-      case 2: return launch_gemm_cfg<kDtype, BN_, ST_, 2>(ma, mb, a, s);                  \
-      case 4: return launch_gemm_cfg<kDtype, BN_, ST_, 4>(ma, mb, a, s);                  \
-      default: return launch_gemm_cfg<kDtype, BN_, ST_, 8>(ma, mb, a, s);                 \
-    }                                                                                     \
+    if (p.small_ring) return launch_split<kDtype, BN_, kSm>(split, ma, mb, a, s);          \
+    return launch_split<kDtype, BN_, ST_>(split, ma, mb, a, s);                             \
   }
   SP24_GEMM_CASE(16, 8)
   SP24_GEMM_CASE(32, 8)

@@ -189,9 +189,11 @@ gemm_sp_kernel(const __grid_constant__ CUtensorMap tmap_a,
   if constexpr (SPLIT > 1) cluster_sync();   // all partials visible cluster-wide
 
   // 2) reduce over the split CTAs (fixed rank order), scale / cast, store.
-  //    CTA `split` owns tokens [split*BN/SPLIT, (split+1)*BN/SPLIT).
-  constexpr int kTokPerCta = BN / SPLIT;
-  const int tok0 = static_cast<int>(split) * kTokPerCta;
+  //    CTA `split` owns tokens [split*BN/SPLIT, (split+1)*BN/SPLIT) (integer
+  //    division: a split that does not divide BN gives some CTAs one token
+  //    more).
+  const int tok0 = static_cast<int>(split) * BN / SPLIT;
+  const int kTokPerCta = (static_cast<int>(split) + 1) * BN / SPLIT - tok0;
   // work item = (token, group of 4 channels); 32 groups per token
   const float sx = (kDtype == SP24_INT8 && args.out_kind != SP24_OUT_INT32) ? *args.s_x : 1.0f;
   const float sy = (kDtype == SP24_INT8 && args.out_kind == SP24_OUT_INT8) ? *args.s_y : 1.0f;

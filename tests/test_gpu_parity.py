@@ -631,7 +631,7 @@ def test_gemm_int8_impls(gemm_impl, out_kind, mnk):
     ok_status()
 
 
-@pytest.mark.parametrize("split", ["1", "2", "4", "8"])
+@pytest.mark.parametrize("split", ["1", "2", "3", "4", "5", "6", "7", "8"])
 @pytest.mark.parametrize("mnk", [(16, 392, 1024), (40, 264, 2048 + 128), (128, 136, 1536)])
 def test_gemm_splitk_forced(split, mnk, monkeypatch):
     # every K split of the split-K kernel (the plan picks few of them)
@@ -653,13 +653,21 @@ def test_gemm_splitk_forced(split, mnk, monkeypatch):
 
 
 # --------------------------------------------- split-K with CTAs sharing SMs
-@pytest.mark.parametrize("mnk", [(16, 11008, 4096), (64, 11008, 4096), (40, 11008, 2048 + 96)])
-def test_gemm_splitk_small_ring(mnk, monkeypatch):
+@pytest.mark.parametrize("case", [(16, 11008, 4096, None), (64, 11008, 4096, None),
+                                  (40, 11008, 2048 + 96, None),
+                                  # forced odd splits: uneven token ownership in the
+                                  # cluster reduction (43/43/42 and 4/3/3/3/3 tokens)
+                                  (128, 11008, 4096, "3"), (100, 11008, 1536, "3"),
+                                  (16, 11008, 4096, "5")])
+def test_gemm_splitk_small_ring(case, monkeypatch):
     # more split CTAs than SMs (several per SM on the small ring): bf16 within
     # the bound, int8 accumulators exact
+    m, n, k, forced = case
     monkeypatch.delenv("SP24_GEMM_IMPL", raising=False)
-    monkeypatch.delenv("SP24_SPLITK", raising=False)
-    m, n, k = mnk
+    if forced:
+        monkeypatch.setenv("SP24_SPLITK", forced)
+    else:
+        monkeypatch.delenv("SP24_SPLITK", raising=False)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     plan = B.sp24_gemm_plan(m, n, k, B.SP24_BF16)
     assert plan["kernel"] == "splitk" and plan["split_k"] > 1 and plan["ctas"] > sms
@@ -787,11 +795,12 @@ def test_gemm_plan_families(monkeypatch):
     assert conv["kernel"] == "single" and conv["ctas"] == sms
     # less than one wave of 128 x 128 tiles (86 for N = 11008): split-K
     assert B.sp24_gemm_plan(128, 11008, 4096, B.SP24_BF16)["kernel"] == "splitk"
-    # 16 tokens, 86 row tiles of 32 stages: split 4 with three CTAs per SM
-    # (24 stages on the busiest SM against 32 unsplit)
+    # 16 tokens, 86 row tiles of 32 stages: split so that several CTAs share
+    # each SM (the exact split depends on how many clusters the GPCs hold)
     dec = B.sp24_gemm_plan(16, 11008, 4096, B.SP24_BF16)
-    assert dec["split_k"] == 4 and dec["ctas"] == 344
-    # 32 row tiles of 86 stages: split 4, one CTA per SM
+    assert dec["split_k"] > 1 and dec["ctas"] == 86 * dec["split_k"] > sms
+    assert dec["cluster"] == dec["split_k"]
+    # 32 row tiles of 86 stages: split 4 fills the SMs once
     dec2 = B.sp24_gemm_plan(16, 4096, 11008, B.SP24_BF16)
     assert dec2["split_k"] == 4 and dec2["ctas"] == 128
     # the one-accumulator 256-token pair tile for the INT8 workload shape
