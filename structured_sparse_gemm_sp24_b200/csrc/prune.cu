@@ -1264,12 +1264,14 @@ __device__ __forceinline__ uint32_t int8_select_key(const uint4* wr, int64_t kve
   return (bucket << 7) | warp_find_bin(h, 128, r2, below2);
 }
 
-// kRegVec > 0: the row (at most 32 * kRegVec vectors) stays in registers
-// between the passes, all its loads in flight at once; 0: any K, the row is
-// read in batches of 8 vectors per lane and again for the second pass.
-constexpr int kInt8RegVec = 16;   // rows up to K = 4096 in registers
+// Two warps per row (4 rows per 256-thread block), each taking every other
+// group of 32 vectors of the row: half h handles vectors lane + 32 * (2 i + h).
+// kHalfVec > 0: a half (at most 32 * kHalfVec vectors) stays in registers
+// between the passes, all its loads in flight at once; 0: any K, the half is
+// read in batches of 8 vectors per lane and again for the output pass.
+constexpr int kInt8HalfVec = 8;   // rows up to K = 4096 in registers
 
-template <int kRegVec>
+template <int kHalfVec>
 __global__ void __launch_bounds__(256) prune_int8_kernel(const uint16_t* __restrict__ w, int64_t n,
                                                          int64_t k, double coverage,
                                                          uint8_t* __restrict__ mask_out,
@@ -1278,81 +1280,103 @@ __global__ void __launch_bounds__(256) prune_int8_kernel(const uint16_t* __restr
                                                          uint8_t* __restrict__ meta) {
   pdl_launch_dependents();
   pdl_wait_prior();
-  __shared__ uint32_t hist[8][256];
+  __shared__ uint32_t hist[4][256];
+  __shared__ uint32_t half_max[8];
+  __shared__ uint32_t row_key[4];
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t wid = threadIdx.x >> 5;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + wid;
+  const uint32_t slot = wid >> 1;        // row within the block
+  const uint32_t half = wid & 1u;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 4 + slot;
+  const bool live = row < n;             // rows >= n: padding of the last 128-row tile
   const int64_t kvec = k / 8;
   const int kblocks = static_cast<int>((k + 127) / 128);
   const int64_t kvec_pad = static_cast<int64_t>(kblocks) * 16;
   // metadata of this row: chunk kb at + kb * 2048, vector bb of the chunk at + bb
   uint8_t* mrow = meta + (row >> 7) * kblocks * 2048 + 16 * (row & 127);
-  if (row >= n) {   // a padding row of the last 128-row tile
-    for (int64_t v = lane; v < kvec_pad; v += 32) mrow[(v >> 4) * 2048 + (v & 15)] = 0x44u;
-    return;
-  }
-  const uint4* wr = reinterpret_cast<const uint4*>(w + row * k);
-  uint4 reg[kRegVec > 0 ? kRegVec : 1];
+  const uint4* wr = reinterpret_cast<const uint4*>(w + (live ? row : 0) * k);
+  // vector of this lane's i-th slot
+  auto vec_of = [&](int64_t i) { return static_cast<int64_t>(lane) + 32 * (2 * i + half); };
+  const int64_t nslots = (kvec + 63) / 64;   // slots per lane over the row
+
+  uint4 reg[kHalfVec > 0 ? kHalfVec : 1];
   uint32_t kmax = 0;
-  if constexpr (kRegVec > 0) {
+  if (live) {
+    if constexpr (kHalfVec > 0) {
 #pragma unroll
-    for (int i = 0; i < kRegVec; ++i) {
-      const int64_t v = lane + 32 * i;
-      reg[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < kRegVec; ++i) kmax = max(kmax, vec_max_key(reg[i]));
-  } else {
-    for (int64_t v0 = lane; v0 < kvec; v0 += 32 * 8) {
-      uint4 b[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t v = v0 + 32 * i;
-        b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < kHalfVec; ++i) {
+        const int64_t v = vec_of(i);
+        reg[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) kmax = max(kmax, vec_max_key(b[i]));
-    }
-  }
+      for (int i = 0; i < kHalfVec; ++i) kmax = max(kmax, vec_max_key(reg[i]));
+    } else {
+      for (int64_t i0 = 0; i0 < nslots; i0 += 8) {
+        uint4 b[8];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+        for (int i = 0; i < 8; ++i) {
+          const int64_t v = vec_of(i0 + i);
+          b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kmax = max(kmax, vec_max_key(b[i]));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+    if (lane == 0) half_max[wid] = kmax;
+  }
+  __syncthreads();
   const uint32_t cnt = static_cast<uint32_t>(kvec * 4);
-  uint32_t key = kmax;
+  uint32_t r = cnt;
   {
     const double rd = ceil(coverage * static_cast<double>(cnt));
-    uint32_t r = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
+    r = rd < 1.0 ? 1u : static_cast<uint32_t>(rd);
     if (r > cnt) r = cnt;
-    if (r < cnt) key = int8_select_key(wr, kvec, r, hist[wid], lane);
   }
-  const float t = __uint_as_float(key << 16);
-  const float s = (cnt == 0 || t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
-  if (lane == 0) s_w[row] = s;
-  const float rs = __frcp_rn(s);
-  uint8_t* mr = mask_out ? mask_out + row * kvec : nullptr;
-  uint32_t* vr = vals + row * kvec;
-  if constexpr (kRegVec > 0) {
+  // the r-th smallest kept key: the row maximum when r = c, else selected by
+  // the row's first warp over the whole row
+  if (live && half == 0) {
+    uint32_t key = max(half_max[2 * slot], half_max[2 * slot + 1]);
+    if (r < cnt) key = int8_select_key(wr, kvec, r, hist[slot], lane);
+    if (lane == 0) row_key[slot] = key;
+  }
+  __syncthreads();
+  if (live) {
+    const uint32_t key = row_key[slot];
+    const float t = __uint_as_float(key << 16);
+    const float s = (cnt == 0 || t == 0.0f) ? 1.0f : __fdiv_rn(t, 127.0f);
+    if (half == 0 && lane == 0) s_w[row] = s;
+    const float rs = __frcp_rn(s);
+    uint8_t* mr = mask_out ? mask_out + row * kvec : nullptr;
+    uint32_t* vr = vals + row * kvec;
+    if constexpr (kHalfVec > 0) {
 #pragma unroll
-    for (int i = 0; i < kRegVec; ++i) {
-      const int64_t v = lane + 32 * i;
-      if (v < kvec) int8_emit(reg[i], v, s, rs, vr, mr, mrow);
-    }
-  } else {
-    for (int64_t v0 = lane; v0 < kvec; v0 += 32 * 8) {
-      uint4 b[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t v = v0 + 32 * i;
-        b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+      for (int i = 0; i < kHalfVec; ++i) {
+        const int64_t v = vec_of(i);
+        if (v < kvec) int8_emit(reg[i], v, s, rs, vr, mr, mrow);
       }
+    } else {
+      for (int64_t i0 = 0; i0 < nslots; i0 += 8) {
+        uint4 b[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int64_t v = v0 + 32 * i;
-        if (v < kvec) int8_emit(b[i], v, s, rs, vr, mr, mrow);
+        for (int i = 0; i < 8; ++i) {
+          const int64_t v = vec_of(i0 + i);
+          b[i] = v < kvec ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int64_t v = vec_of(i0 + i);
+          if (v < kvec) int8_emit(b[i], v, s, rs, vr, mr, mrow);
+        }
       }
     }
   }
-  // positions >= K of the last 128-position chunk: the padding pattern
-  for (int64_t v = kvec + lane; v < kvec_pad; v += 32) mrow[(v >> 4) * 2048 + (v & 15)] = 0x44u;
+  // metadata padding: positions >= K of the last 128-position chunk, and
+  // whole rows >= n of the last 128-row tile
+  const int64_t pad0 = live ? kvec : 0;
+  for (int64_t v = pad0 + lane + 32 * half; v < kvec_pad; v += 64)
+    mrow[(v >> 4) * 2048 + (v & 15)] = 0x44u;
 }
 
 // ------------------------------------------- Wanda prune without allocation
@@ -1707,9 +1731,9 @@ sp24_status sp24_prune_compress_int8(const void* W, int64_t N, int64_t K, double
   if (N > (int64_t(1) << 31) || K > (int64_t(1) << 31)) return SP24_ERR_UNSUPPORTED;
   SP24_TRY(check_device());
   const int64_t n_pad = (N + 127) / 128 * 128;   // padding rows of the last tile too
-  const dim3 grid(static_cast<unsigned>(n_pad / 8));
-  if (K / 8 <= 32 * kInt8RegVec)
-    return launch_kernel(prune_int8_kernel<kInt8RegVec>, grid, dim3(256), 0, as_stream(stream),
+  const dim3 grid(static_cast<unsigned>(n_pad / 4));
+  if (K / 8 <= 64 * kInt8HalfVec)
+    return launch_kernel(prune_int8_kernel<kInt8HalfVec>, grid, dim3(256), 0, as_stream(stream),
                          1, static_cast<const uint16_t*>(W), N, K, coverage, mask_out, s_w,
                          static_cast<uint32_t*>(vals), static_cast<uint8_t*>(meta));
   return launch_kernel(prune_int8_kernel<0>, grid, dim3(256), 0, as_stream(stream), 1,
