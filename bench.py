@@ -232,6 +232,32 @@ class Runner:
             self.gemm_call()
         rec(3)
 
+    def prep_call(self):
+        """The step's work before the GEMM (prune / compress, and for INT8 the
+        weight conversion, activation scale and quantisation)."""
+        wl = self.wl
+        if wl.int8:
+            B.sp24_prune_compress_int8(self.W, 0.9999, self.mask2, self.s_w, self.vals,
+                                       self.meta)
+            B.sp24_act_scale(self.X, 0.9999, self.s_x, self.act_ws)
+            B.sp24_quantize(self.X, self.s_x, self.Xq)
+        elif self.wanda and wl.progressive:
+            B.sp24_prune_progressive(self.W, self.Xc, B.SP24_WANDA, self.mask1, self.mask2,
+                                     self.vals, self.meta, self.ws)
+        elif self.wanda:
+            B.sp24_prune(self.W, self.Xc, B.SP24_WANDA, 2, None, self.mask1, self.ws)
+            B.sp24_prune_compress(self.W, B.SP24_WANDA, self.ws, None, None, B.SP24_BF16,
+                                  None, self.vals, self.meta)
+        else:
+            B.sp24_prune_compress(self.W, B.SP24_MAGNITUDE, None, None, None, B.SP24_BF16, None,
+                                  self.vals, self.meta)
+
+    def prep_bytes(self) -> float:
+        """Algorithmic bytes of prep_call."""
+        if self.wl.int8:
+            return self.prune_bytes() + self.compress_bytes()
+        return self.compress_bytes()
+
     def gemm_call(self):
         """The step's GEMM (its operands are the step's earlier outputs)."""
         if self.wl.int8:
@@ -494,6 +520,7 @@ def measure_config(name, device, flush, peaks, steps):
     # how it runs between other kernels of a model, without the event nodes
     # of the stage timing
     b2b_ms = time_graph(lambda: [runner.gemm_call() for _ in range(5)], flush) / 5
+    prep_b2b_ms = time_graph(lambda: [runner.prep_call() for _ in range(5)], flush) / 5
     if B.sp24_device_status() != B.SP24_OK:
         raise SystemExit(f"device status not OK after config {name}")
     gemm_ms, comp_ms = statistics.median(gemm), statistics.median(comp)
@@ -518,6 +545,10 @@ def measure_config(name, device, flush, peaks, steps):
                            "frac_hbm": c_gbs / peaks["hbm_gbs"],
                            "prune_us": 1e3 * statistics.median(prune)},
     }
+    prep_gbs = runner.prep_bytes() / (prep_b2b_ms * 1e-3) / 1e9
+    out["prune_compress"]["back_to_back_us"] = 1e3 * prep_b2b_ms
+    out["prune_compress"]["back_to_back_gbs"] = prep_gbs
+    out["prune_compress"]["frac_hbm_back_to_back"] = prep_gbs / peaks["hbm_gbs"]
     if wl.int8:
         # INT8: the first stage is the one-pass weight conversion, the second
         # the activation side (scale and quantisation)
