@@ -867,7 +867,7 @@ __global__ void __launch_bounds__(256) act_bracket(const float4* __restrict__ x,
   __syncthreads();
   const uint32_t lo = ws->lo, hi = ws->hi;
   uint32_t below = 0;
-  constexpr int kU = 4;   // float4 loads in flight per thread
+  constexpr int kU = 8;   // float4 loads in flight per thread
   const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t v = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   for (; v + (kU - 1) * step < nvec; v += kU * step) {
