@@ -447,6 +447,22 @@ def count_step_kernels(runner):
         return None
 
 
+class nvtx_range:
+    """An NVTX range around a phase of the bench (timeline tools show the
+    phases; nothing is recorded without one attached)."""
+
+    def __init__(self, name: str):
+        self.name = name
+
+    def __enter__(self):
+        torch.cuda.nvtx.range_push(self.name)
+        return self
+
+    def __exit__(self, *exc):
+        torch.cuda.nvtx.range_pop()
+        return False
+
+
 def max_over_ranks(value: float, device) -> float:
     """The maximum of a per-rank time over all ranks (every rank calls it at the
     same point; all_reduce MAX), or the value itself in a single process."""
@@ -891,7 +907,7 @@ def main(argv=None):
         print(f"bench: step graph holds {counted} kernels, expected "
               f"{runner.launches_per_step()}", file=sys.stderr)
     barrier()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local) as clk, nvtx_range(f"sp24 timed steps: {wl.name}"):
         tot, prune, comp, gemm = time_steps(runner, args.steps, flush,
                                             use_graph=not args.no_graph, stage_steps=50)
     barrier()
@@ -900,8 +916,9 @@ def main(argv=None):
     value = job_tflops(world, args.steps, runner.flops(), total_ms)
 
     e2e_steps = max(3, min(args.steps, 50 if wl.N * wl.K < (1 << 26) else 10))
-    serial_ms, h2d, d2h = time_e2e(runner, e2e_steps)
-    e2e_ms = time_e2e_pipelined(runner, e2e_steps)
+    with nvtx_range("sp24 end to end (serial, then pipelined)"):
+        serial_ms, h2d, d2h = time_e2e(runner, e2e_steps)
+        e2e_ms = time_e2e_pipelined(runner, e2e_steps)
     serial_ms = max_over_ranks(serial_ms, device)
     e2e_ms = max_over_ranks(e2e_ms, device)
     e2e_value = job_tflops(world, 1, runner.flops(), e2e_ms)
@@ -963,9 +980,11 @@ def main(argv=None):
     del runner
     torch.cuda.empty_cache()
     if world == 1 and not args.no_configs:
-        line["configs"] = [measure_config(n, device, flush, peaks, args.config_steps)
-                           for n in CONFIG_WORKLOADS if n != wl.name]
-        line["extras"] = measure_extras(device, flush, peaks)
+        with nvtx_range("sp24 configured workloads"):
+            line["configs"] = [measure_config(n, device, flush, peaks, args.config_steps)
+                               for n in CONFIG_WORKLOADS if n != wl.name]
+        with nvtx_range("sp24 extra rows"):
+            line["extras"] = measure_extras(device, flush, peaks)
     if world == 1 and not args.no_cpu_baseline:
         flops, secs, sample, cores = oracle_sample(wl, args.cpu_budget)
         line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": cores,

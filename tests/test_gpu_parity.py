@@ -501,6 +501,28 @@ def test_gemm_bf16_deterministic_split():
         assert torch.equal(y1, y2)
 
 
+def test_compressed_weight_file_round_trip(tmp_path):
+    # compress once, save, load back onto the device: the GEMM on the loaded
+    # weight gives the same bits (bf16) and the same accumulators (int8)
+    from structured_sparse_gemm_sp24_b200 import artifact as A
+    w = I.llm_proj(1024, 2048, 64)
+    Wd, Xd = w.W.cuda(), w.X.cuda()
+    vals, meta = P.prune_compress(Wd)
+    A.save_compressed(str(tmp_path / "w.sp24"), vals, meta, w.N, w.K, B.SP24_BF16)
+    cw = A.load_compressed(str(tmp_path / "w.sp24"), "cuda")
+    assert torch.equal(P.gemm(Xd, cw.vals, cw.meta, cw.n), P.gemm(Xd, vals, meta, w.N))
+    v8, m8, s_w = P.prune_compress_int8(Wd)
+    A.save_compressed(str(tmp_path / "w8.sp24"), v8, m8, w.N, w.K, B.SP24_INT8, s_w)
+    c8 = A.load_compressed(str(tmp_path / "w8.sp24"), "cuda")
+    xf = I.normal_f32((64, w.K), 1.0, seed=9).cuda()
+    s_x = P.act_scale(xf)
+    xq = P.quantize(xf, s_x)
+    a = P.gemm(xq, c8.vals, c8.meta, c8.n, B.SP24_INT8, s_x, c8.s_w, B.SP24_OUT_INT32)
+    b = P.gemm(xq, v8, m8, w.N, B.SP24_INT8, s_x, s_w, B.SP24_OUT_INT32)
+    assert torch.equal(a, b)
+    ok_status()
+
+
 def test_gemm_empty_is_noop():
     W = I.normal_bf16((64, 128), 1.0, seed=1).cuda()
     mask = P.prune(W, B.SP24_MAGNITUDE, 2)
