@@ -385,10 +385,13 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
     }
     const bool ready = mbar_wait(&full[st], (i / kStreamStages) & 1u);
     const bool kv_ok = kv < kvec && ready;
+    double zero_sc[8];   // progressive Wanda: the score of a zero weight, 0 * n_j
     if constexpr (kWanda) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
+      for (int e = 0; e < 8; ++e) {
         nrm[e] = reinterpret_cast<const double*>(sb + kWTile + kMTile)[bb * 8 + e];
+        if constexpr (kProg) zero_sc[e] = __dmul_rn(0.0, nrm[e]);
+      }
     }
     // per-thread bases: chunk row m0 + 32 j is +8192 bytes of the W tile,
     // +512 bytes of the mask tile, of the metadata chunk (both layouts) and
@@ -421,8 +424,21 @@ stream_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ 
           // stage 1 keeps 3 of 4; stage 2 keeps 2 of 4 of what stage 1 kept
           uint32_t k3;
           if constexpr (kWanda) {
-            k3 = mask_byte<true>(q, 0xFFu, nrm, 3);
-            keep = mask_byte<true>(q, k3, nrm, 2);
+            // the products |w| * n_j once; stage 2 scores a dropped position
+            // as a zero weight (0 * n_j, as mask_byte with mask_in does)
+            const uint32_t words[4] = {q.x, q.y, q.z, q.w};
+            double sc[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t bits = (e & 1) ? (words[e / 2] >> 16) : (words[e / 2] & 0xFFFFu);
+              sc[e] = __dmul_rn(fabs(bf16_to_double(bits)), nrm[e]);
+            }
+            k3 = keep_nibble(sc[0], sc[1], sc[2], sc[3], 3) |
+                 (keep_nibble(sc[4], sc[5], sc[6], sc[7], 3) << 4);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc[e] = ((k3 >> e) & 1u) ? sc[e] : zero_sc[e];
+            keep = keep_nibble(sc[0], sc[1], sc[2], sc[3], 2) |
+                   (keep_nibble(sc[4], sc[5], sc[6], sc[7], 2) << 4);
           } else {
             k3 = keep_nibble_mag<false>(q.x, q.y, 0xFu, 3) |
                  (keep_nibble_mag<false>(q.z, q.w, 0xFu, 3) << 4);
