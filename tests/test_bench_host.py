@@ -115,3 +115,33 @@ def test_single_process_reduction_is_identity():
     import torch
     assert bench.max_over_ranks(3.5, torch.device("cpu")) == 3.5
     assert bench.job_tflops(1, 10, 1e12, 10.0) == 1000.0
+
+
+def test_back_to_back_timings_run_the_step_work(monkeypatch):
+    # the per-configuration "back to back" figures time prep_call() and
+    # gemm_call(); together they must issue exactly the library calls of one
+    # step, in order.  The launching entry points are replaced by recorders
+    # (no GPU), the size queries stay the library's own.
+    import torch
+    from structured_sparse_gemm_sp24_b200 import build as sp24_build
+    from structured_sparse_gemm_sp24_b200 import inputs as I
+    from structured_sparse_gemm_sp24_b200 import sp24 as B
+    sp24_build.build()
+    B.lib()
+    calls = []
+    for name in ["sp24_prune", "sp24_prune_compress", "sp24_prune_progressive",
+                 "sp24_prune_compress_int8", "sp24_act_scale", "sp24_quantize", "sp24_gemm"]:
+        monkeypatch.setattr(B, name, (lambda n: lambda *a, **k: calls.append(n))(name))
+    workloads = [I.tiny(), I.bert_fc1(), I.int8_long_tail(M=64, N=256, K=256)]
+    for wl in workloads:
+        r = bench.Runner(wl, torch.device("cpu"))
+        calls.clear()
+        r.step()
+        step_calls = list(calls)
+        calls.clear()
+        r.prep_call()
+        r.gemm_call()
+        assert calls == step_calls, (wl.name, calls, step_calls)
+        assert step_calls[-1] == "sp24_gemm"
+        # the prep stage's bytes cover what its calls move
+        assert r.prep_bytes() >= r.compress_bytes() > 0
