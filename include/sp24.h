@@ -320,8 +320,10 @@ sp24_status sp24_gemm(const void* X, int64_t M, int64_t K, const void* vals,
  * current device (the pages fix no kernel design; this reports the one this
  * library chose, for profiling and tests).  Fills *plan; allocates nothing
  * and launches nothing.  The SP24_GEMM_IMPL environment variable, if set
- * (pair256, pair240, pair224, pair192, pair128, single), overrides the
- * persistent-kernel choice exactly as it does for sp24_gemm.
+ * (pair256, pair240, pair224, pair192, pair128, single, splitk), overrides
+ * the kernel choice exactly as it does for sp24_gemm, and SP24_SPLITK (1..8)
+ * the split-K kernel's split (tuning overrides; results never depend on
+ * them beyond float32 summation order).
  *   kernel:        "splitk" (few tokens or tiles: K split across a cluster),
  *                  "single" (persistent, one 128 x 128 tile per SM at a time),
  *                  "pairNNN" (persistent, a CTA pair on two SMs computes
